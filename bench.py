@@ -1,0 +1,494 @@
+#!/usr/bin/env python
+"""Benchmark of the LLM.int8() mixed-precision decomposition matmul on B200.
+
+Default workload: the 7B decode GEMV sweep -- X fp16 [T, 4096] for
+T = 1, 2, 4, 8, 16 against W [11008, 4096], four systematic outlier dims,
+threshold 6.0.  One step = the five llmint8_matmul calls, each on its own
+weight matrix (five independent layers, so no call finds its weights in L2).
+L2 is flushed (256 MiB write) before every timed step.  Metric: algorithmic
+HBM bytes / time (Wq + Wscale + outlier columns of W + X + Y).
+
+Prefill workloads (--workload 7b_prefill | 13b_up | 70b_up) report effective
+TOPS = 2 T N K / time; at N=1 they are also measured by default and reported
+under "also".
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+--impl reference times the CPU oracle (the plain C statement of the method
+that the tests check the kernels against) on the host cores, on a bounded
+sample of the same workload.  Under torchrun, rank 0 alone runs it.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from int8_mixed_precision_outlier_b200 import synth  # noqa: E402
+
+METRIC = "LLM.int8 matmul effective TOPS (2TNK/s) vs int8 TC peak; decode GEMV HBM GB/s"
+FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+INT8_PER_BF16 = 2.0  # nominal dense ratio: 4.5 POPS int8 / 2.25 PFLOPS bf16
+THRESHOLD = 6.0
+FLUSH_BYTES = 256 << 20
+DECODE_TS = (1, 2, 4, 8, 16)
+
+
+# ----------------------------------------------------------------- helpers
+
+def load_peaks() -> dict:
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                "source": "measured"}
+    except Exception:
+        return dict(FALLBACK, source="fallback")
+
+
+def source_digest() -> str:
+    """sha256 over the CUDA sources: a recorded ncu traffic figure is only used
+    while the kernels it was measured on are unchanged."""
+    import glob
+    import hashlib
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "int8_mixed_precision_outlier_b200", "csrc")
+    for f in sorted(glob.glob(os.path.join(csrc, "*.cu*"))):
+        with open(f, "rb") as fh:
+            h.update(os.path.basename(f).encode() + b"\0" + fh.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(workload: str, kernel: str):
+    """dram bytes per launch of `kernel` on `workload` from profiles/traffic.txt
+    (lines: workload kernel source_digest bytes_per_launch), or None."""
+    p = os.path.join(ROOT, "profiles", "traffic.txt")
+    if not os.path.exists(p):
+        return None
+    digest = source_digest()
+    with open(p) as f:
+        for line in f:
+            parts = line.split("#", 1)[0].split()
+            if len(parts) == 4 and parts[0] == workload and parts[1] == kernel and parts[2] == digest:
+                return float(parts[3])
+    return None
+
+
+def dist_env():
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def reduce_max(value: float, world: int) -> float:
+    """Max over ranks (the slowest rank sets the job's time)."""
+    if world == 1:
+        return float(value)
+    import torch
+    import torch.distributed as dist
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([float(value)], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def reduce_sum(value: float, world: int) -> float:
+    if world == 1:
+        return float(value)
+    import torch
+    import torch.distributed as dist
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([float(value)], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+           0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+           0x2: "applications_clocks_setting", 0x10: "sync_boost"}
+
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML while the timed region runs."""
+
+    def __init__(self, cuda_index: int, period_s: float = 0.01):
+        self.samples, self.reasons, self.max_mhz, self.ok = [], 0, None, False
+        self._stop = threading.Event()
+        self._period = period_s
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
+            idx = cuda_index
+            if vis and all(v.strip().isdigit() for v in vis.split(",")):
+                idx = int(vis.split(",")[cuda_index])
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(idx)
+            self._nv = pynvml
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.ok = False
+        self._t = threading.Thread(target=self._run, daemon=True)
+
+    def _run(self):
+        nv = self._nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                self.reasons |= nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+            except Exception:
+                pass
+            time.sleep(self._period)
+
+    def __enter__(self):
+        if self.ok:
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self.ok:
+            self._t.join()
+
+    def summary(self) -> dict:
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0,
+                    "note": "NVML sampling unavailable"}
+        names = [n for bit, n in REASONS.items() if self.reasons & bit]
+        return {"sm_mhz": float(statistics.median(self.samples)), "sm_max_mhz": self.max_mhz,
+                "reasons": names, "samples": len(self.samples)}
+
+
+# ----------------------------------------------------------------- workloads
+
+class Workload:
+    """Device-resident inputs and the list of calls one step makes."""
+
+    def __init__(self, name: str, device, seed: int = 0, taus=None):
+        import torch
+        import int8_mixed_precision_outlier_b200 as L
+        self.L, self.name, self.device = L, name, device
+        cfg = synth.WORKLOADS[name]
+        self.K, self.N = cfg["K"], cfg["N"]
+        self.calls = []  # dicts: X, Wq, sw, W, Y, tau, T, host data
+        if name == "7b_decode":
+            ws = L.alloc_workspace(16, self.N, self.K, device)
+            for layer, T in enumerate(DECODE_TS):
+                w = synth.workload(name, seed=seed, T=T, layer=layer)
+                self._add(w, T, THRESHOLD, ws)
+            self.unit, self.kind = "GB/s", "hbm"
+        else:
+            w = synth.workload(name, seed=seed)
+            ws = L.alloc_workspace(w["T"], self.N, self.K, device)
+            taus = taus if taus is not None else ((THRESHOLD,) if name != "70b_up" else w["thresholds"])
+            Wd = None
+            for tau in taus:
+                Wd = self._add(w, w["T"], tau, ws, share_w=Wd)
+            self.unit, self.kind = "TOPS", "tensor"
+        torch.cuda.synchronize()
+        self.bytes_per_step = sum(c["bytes"] for c in self.calls)
+        self.ops_per_step = sum(c["ops"] for c in self.calls)
+        self.launches_per_step = sum(2 if c["T"] <= 16 else 4 for c in self.calls)
+
+    def _add(self, w, T, tau, ws, share_w=None):
+        import torch
+        L = self.L
+        X = torch.from_numpy(w["X"]).to(self.device)
+        if share_w is None:
+            W = torch.from_numpy(w["W"]).to(self.device)
+            Wq, sw = L.llmint8_quantize_weight(W)
+            share_w = (W, Wq, sw)
+        W, Wq, sw = share_w
+        Y = torch.empty((T, self.N), dtype=torch.float16, device=self.device)
+        _, _, idx = L.llmint8_detect_quantize(X, tau)
+        nO = int(idx.numel())
+        K, N = self.K, self.N
+        algo_bytes = N * K + 4 * N + 2 * N * nO + 2 * T * K + 2 * T * N
+        self.calls.append(dict(X=X, W=W, Wq=Wq, sw=sw, Y=Y, ws=ws, tau=tau, T=T, nO=nO,
+                               bytes=algo_bytes, ops=2 * T * N * K, host_X=w["X"], host_W=w["W"]))
+        return share_w
+
+    def step(self):
+        L = self.L
+        for c in self.calls:
+            L.llmint8_matmul(c["X"], c["Wq"], c["sw"], c["W"], c["tau"], c["ws"], c["Y"])
+
+    def metric_value(self, seconds: float, steps: int) -> float:
+        if self.unit == "GB/s":
+            return self.bytes_per_step * steps / seconds / 1e9
+        return self.ops_per_step * steps / seconds / 1e12
+
+
+def time_steps(wl: Workload, steps: int, warmup: int, world: int, flush, run=None):
+    """Events around each step on the launching stream; L2 flushed before each."""
+    import torch
+    run = run or wl.step
+    for _ in range(warmup):
+        flush.zero_()
+        run()
+    stream = torch.cuda.current_stream()
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    barrier(world)
+    torch.cuda.synchronize()
+    sampler = ClockSampler(torch.cuda.current_device())
+    with sampler:
+        for i in range(steps):
+            flush.zero_()
+            starts[i].record(stream)
+            run()
+            ends[i].record(stream)
+        torch.cuda.synchronize()
+    barrier(world)
+    total_ms = sum(s.elapsed_time(e) for s, e in zip(starts, ends))
+    return total_ms, sampler.summary()
+
+
+def time_main_kernel(wl: Workload, steps: int, flush) -> tuple[float, int]:
+    """Average duration of the main kernel (GEMV or GEMM) per launch, CUDA events."""
+    import torch
+    L = wl.L
+    pairs = []
+    for _ in range(steps):
+        flush.zero_()
+        for c in wl.calls:
+            b = torch.cuda.Event(enable_timing=True)
+            e = torch.cuda.Event(enable_timing=True)
+            L.llmint8_matmul_profile(c["X"], c["Wq"], c["sw"], c["W"], c["tau"], c["ws"], c["Y"], b, e)
+            pairs.append((b, e, c))
+    torch.cuda.synchronize()
+    total = sum(b.elapsed_time(e) for b, e, _ in pairs)
+    algo = sum(c["bytes"] if wl.unit == "GB/s" else c["ops"] for _, _, c in pairs)
+    return total / len(pairs), algo / len(pairs)
+
+
+def main_kernel_name(wl: Workload) -> str:
+    return "gemv_kernel" if wl.unit == "GB/s" else "gemm_kernel"
+
+
+def roofline(wl: Workload, kern_ms: float, algo_per_launch: float, peaks: dict, traffic=None) -> dict:
+    if wl.unit == "GB/s":
+        achieved = algo_per_launch / (kern_ms * 1e-3) / 1e9
+        peak = peaks["hbm_gbs"]
+        return {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                "frac": round(achieved / peak, 4), "traffic": traffic,
+                "kernel": "gemv_kernel (stream-K tcgen05, swap-AB)",
+                "peak_source": f"{peaks['source']} hbm_gbs (copy, burst)",
+                "algo_bytes_per_launch": int(algo_per_launch), "ms_per_launch": round(kern_ms, 5)}
+    achieved = algo_per_launch / (kern_ms * 1e-3) / 1e12
+    peak = peaks["bf16_tflops"] * INT8_PER_BF16
+    return {"bound": "tensor", "achieved": round(achieved, 1), "peak": round(peak, 1), "unit": "TOPS",
+            "frac": round(achieved / peak, 4), "traffic": traffic,
+            "kernel": "gemm_kernel (tcgen05 kind::i8 + kind::f16)",
+            "peak_source": f"{peaks['source']} bf16_tflops (burst) x 2 (nominal int8/bf16 ratio)",
+            "algo_ops_per_launch": int(algo_per_launch), "ms_per_launch": round(kern_ms, 5)}
+
+
+def e2e_steps(wl: Workload, steps: int, warmup: int, flush) -> dict:
+    """The public call with host buffers: pinned H2D of X, the matmul, D2H of Y."""
+    import torch
+    L = wl.L
+    hx = [torch.from_numpy(c["host_X"]).pin_memory() for c in wl.calls]
+    hy = [torch.empty(c["Y"].shape, dtype=torch.float16).pin_memory() for c in wl.calls]
+
+    def run():
+        for c, x, y in zip(wl.calls, hx, hy):
+            c["X"].copy_(x, non_blocking=True)
+            L.llmint8_matmul(c["X"], c["Wq"], c["sw"], c["W"], c["tau"], c["ws"], c["Y"])
+            y.copy_(c["Y"], non_blocking=True)
+
+    total_ms, _ = time_steps(wl, steps, warmup, 1, flush, run=run)
+    h2d = sum(x.numel() * 2 for x in hx)
+    d2h = sum(y.numel() * 2 for y in hy)
+    return {"value": round(wl.metric_value(total_ms * 1e-3, steps), 2), "unit": wl.unit,
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "ms_per_step": round(total_ms / steps, 5)}
+
+
+# ----------------------------------------------------------------- CPU oracle
+
+def oracle_sample(name: str, seed: int = 0):
+    """Oracle inputs and one step's calls, on a bounded sample of the workload.
+
+    Decode: the full step (five calls).  Prefill: the first `rows` rows of X
+    against the full W (detection and scales then cover those rows only).
+    """
+    from oracle import oracle as O
+    cfg = synth.WORKLOADS[name]
+    calls = []
+    if name == "7b_decode":
+        for layer, T in enumerate(DECODE_TS):
+            w = synth.workload(name, seed=seed, T=T, layer=layer)
+            Wq, sw = O.quantize_weight(w["W"])
+            nO = int(O.compact(O.detect_outliers(w["X"], THRESHOLD)).size)
+            calls.append((w["X"], Wq, sw, w["W"], THRESHOLD,
+                          cfg["N"] * cfg["K"] + 4 * cfg["N"] + 2 * cfg["N"] * nO +
+                          2 * T * cfg["K"] + 2 * T * cfg["N"], 2 * T * cfg["N"] * cfg["K"]))
+        return calls, "full step: 5 calls, T=1,2,4,8,16, full N and K", "GB/s"
+    w = synth.workload(name, seed=seed)
+    rows = 16 if name == "70b_up" else 32
+    Xs = np.ascontiguousarray(w["X"][:rows])
+    Wq, sw = O.quantize_weight(w["W"])
+    T, N, K = rows, cfg["N"], cfg["K"]
+    calls.append((Xs, Wq, sw, w["W"], THRESHOLD, 0, 2 * T * N * K))
+    return calls, f"first {rows} rows of X against the full W, tau=6 (ops scaled to those rows)", "TOPS"
+
+
+def run_oracle(calls, unit, steps: int, budget_s: float):
+    from oracle import oracle as O
+    done, t0 = 0, time.perf_counter()
+    while done < steps:
+        for X, Wq, sw, W, tau, _, _ in calls:
+            O.matmul(X, Wq, sw, W, tau)
+        done += 1
+        if time.perf_counter() - t0 > budget_s:
+            break
+    dt = time.perf_counter() - t0
+    per = sum(c[5] for c in calls) if unit == "GB/s" else sum(c[6] for c in calls)
+    value = per * done / dt / (1e9 if unit == "GB/s" else 1e12)
+    return value, done, dt, O.num_threads()
+
+
+# ----------------------------------------------------------------- arms
+
+def run_reference(args):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return 0
+    calls, sample, unit = oracle_sample(args.workload)
+    run_oracle(calls, unit, max(1, min(args.warmup, 1)), 1e9)  # warm caches/threads
+    value, done, dt, cores = run_oracle(calls, unit, args.steps, args.ref_budget_s)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": unit,
+        "n_gpus": args.gpus, "steps": done, "warmup": args.warmup,
+        "ms_per_step": round(dt / done * 1e3, 3), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "int8", "data": "synthetic",
+        "config": workload_config(args.workload),
+        "cpu_baseline": {"value": round(value, 4), "unit": unit, "cores": cores, "kind": "oracle",
+                         "sample": sample + f"; {done} steps in {dt:.1f} s"},
+        "e2e": {"value": round(value, 4), "unit": unit, "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def workload_config(name: str) -> dict:
+    cfg = synth.WORKLOADS[name]
+    d = {"workload": name, "T": list(cfg["T"]) if isinstance(cfg["T"], tuple) else cfg["T"],
+         "N": cfg["N"], "K": cfg["K"], "threshold": THRESHOLD if name != "70b_up" else
+         list(cfg["thresholds"]), "l2": "flushed before every step (256 MiB write)",
+         "parallelism": "replicas (one independent problem per GPU)"}
+    if name == "7b_decode":
+        d["layers_per_step"] = len(DECODE_TS)
+    return d
+
+
+def run_ours(args):
+    import torch
+    rank, world, local = dist_env()
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    device = torch.device("cuda", torch.cuda.current_device())
+    from int8_mixed_precision_outlier_b200 import _build
+    if rank == 0:
+        _build.build()
+    barrier(world)
+    import int8_mixed_precision_outlier_b200 as L
+    L.load_library()
+    peaks = load_peaks()
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=device)
+
+    wl = Workload(args.workload, device, seed=rank)
+    total_ms, clocks = time_steps(wl, args.steps, args.warmup, world, flush)
+    t_max = reduce_max(total_ms, world)
+    units = reduce_sum((wl.bytes_per_step if wl.unit == "GB/s" else wl.ops_per_step) * args.steps, world)
+    value = units / (t_max * 1e-3) / (1e9 if wl.unit == "GB/s" else 1e12)
+    status = L.llmint8_sync_status()
+    kern_ms, algo = time_main_kernel(wl, max(3, args.steps // 4), flush)
+    line = {
+        "metric": METRIC, "value": round(value, 3), "unit": wl.unit, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(t_max / args.steps, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int8",
+        "data": "synthetic", "config": workload_config(args.workload),
+        "roofline": roofline(wl, kern_ms, algo, peaks,
+                             traffic=recorded_traffic(args.workload, main_kernel_name(wl))),
+        "gpu_launches": wl.launches_per_step * args.steps,
+        "clocks": clocks, "device_status": L.llmint8_status_string(status),
+    }
+    if rank == 0 and world == 1:
+        line["e2e"] = e2e_steps(wl, args.steps, args.warmup, flush)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        calls, sample, unit = oracle_sample(args.workload)
+        v, done, dt, cores = run_oracle(calls, unit, 1000, args.cpu_budget_s)
+        line["cpu_baseline"] = {"value": round(v, 4), "unit": unit, "cores": cores, "kind": "oracle",
+                                "sample": sample + f"; {done} steps in {dt:.1f} s"}
+    if rank == 0 and world == 1 and args.also:
+        also = []
+        for name in ("7b_prefill", "13b_up", "70b_up"):
+            if name == args.workload:
+                continue
+            w2 = Workload(name, device, taus=(THRESHOLD,))
+            ms, ck = time_steps(w2, args.also_steps, 3, 1, flush)
+            km, ka = time_main_kernel(w2, 3, flush)
+            also.append({"workload": name, "value": round(w2.metric_value(ms * 1e-3, args.also_steps), 2),
+                         "unit": w2.unit, "ms_per_call": round(ms / args.also_steps, 4),
+                         "n_outliers": w2.calls[0]["nO"], "threshold": THRESHOLD,
+                         "roofline": roofline(w2, km, ka, peaks,
+                                              traffic=recorded_traffic(name, main_kernel_name(w2))),
+                         "sm_mhz": ck.get("sm_mhz")})
+            del w2
+            torch.cuda.empty_cache()
+        line["also"] = also
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--workload", choices=tuple(synth.WORKLOADS), default="7b_decode")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-also", dest="also", action="store_false")
+    ap.add_argument("--also-steps", type=int, default=20)
+    ap.add_argument("--cpu-budget-s", type=float, default=15.0)
+    ap.add_argument("--ref-budget-s", type=float, default=120.0)
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.workload == "tiny":
+        ap.error("the tiny configuration is a parity case, not a bench workload")
+    return run_reference(args) if args.impl == "reference" else run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

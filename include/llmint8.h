@@ -1,0 +1,173 @@
+/*
+ * llmint8.h -- C ABI of the B200 (sm_100a) LLM.int8() mixed-precision
+ * decomposition matmul  Y = X * W^T.
+ *
+ * The method (pages on LLM quantization; titles as printed, sections theirs):
+ *   'LLM quantization, part 2' (hncyxsy.com/news/230290) §2.1: vector-wise
+ *     quantization (one int8 scale per output feature of W) and mixed-precision
+ *     decomposition: feature dims whose activation magnitude reaches a
+ *     threshold (usually 6.0) are outliers; those columns of X and W are
+ *     multiplied in fp16, all other columns as an int8 matrix product, and the
+ *     two partial results are added.
+ *   '三、模型量化' (lowentro.cn) Q2: symmetric int8, q = round(r/s),
+ *     s = max|r| / 127, dequantised r' = s*q.  Q4: the same decomposition.
+ *   '量化压缩实战：INT8 / INT4 / AWQ / GPTQ 全面对比' (tqpw.cn) §2.1: absmax
+ *     recipe (scale = max_val/127, round, clip) and its worked example.
+ *
+ * Conventions for every entry point
+ *   - Layouts: X fp16 [T][K] row-major, W fp16 [N][K] row-major (out-features
+ *     x in-features), Wq int8 [N][K], Y fp16 [T][N]; all contiguous.
+ *   - fp16 buffers are passed as `void*` holding IEEE binary16 values.
+ *   - Every pointer is a DEVICE pointer on the current CUDA device unless the
+ *     comment says host.  The caller owns all memory; the library allocates
+ *     nothing on these calls and keeps no pointer after a call returns.
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Calls are
+ *     asynchronous on it; outputs are ready when the stream reaches them.
+ *   - Alignment: X, W, Wq, Y, workspace 16-byte aligned; K % 16 == 0.
+ *   - Return value: an llmint8_status.  Argument and launch errors return at
+ *     once and launch nothing.  A device-side fault detected by a kernel (a
+ *     bounded wait that ran out) is recorded in a per-device error word and
+ *     reported by llmint8_sync_status().
+ *   - Requires an sm_100 device (B200); otherwise LLMINT8_ERR_UNSUPPORTED_ARCH.
+ */
+#ifndef LLMINT8_H
+#define LLMINT8_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define LLMINT8_API __attribute__((visibility("default")))
+#else
+#define LLMINT8_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  LLMINT8_OK = 0,
+  LLMINT8_ERR_INVALID_ARG = -1,      /* null pointer, bad size, NaN threshold, bad path   */
+  LLMINT8_ERR_ALIGNMENT = -2,        /* pointer not 16-byte aligned or K % 16 != 0         */
+  LLMINT8_ERR_UNSUPPORTED_ARCH = -3, /* current device is not compute capability 10.x      */
+  LLMINT8_ERR_WORKSPACE = -4,        /* workspace smaller than llmint8_workspace_bytes()   */
+  LLMINT8_ERR_CUDA = -5,             /* a CUDA runtime call failed (launch, attribute ...) */
+  LLMINT8_ERR_TIMEOUT = -6,          /* a kernel's bounded wait ran out (device error word) */
+  LLMINT8_ERR_UNIMPLEMENTED = -7
+} llmint8_status;
+
+/* Kernel path of llmint8_matmul.  AUTO takes GEMV for T <= 16, else GEMM. */
+enum {
+  LLMINT8_PATH_AUTO = 0,
+  LLMINT8_PATH_GEMV = 1, /* decode: weight-streaming split-K tcgen05 (T <= 16 only)     */
+  LLMINT8_PATH_GEMM = 2  /* prefill: TMA-fed tcgen05 int8 GEMM + fp16 outlier GEMM      */
+};
+
+/* Largest T the decode path takes. */
+#define LLMINT8_GEMV_MAX_T 16
+
+/* Static text for a status code (host only, never NULL). */
+LLMINT8_API const char* llmint8_status_string(int status);
+
+/* Library version, major*10000 + minor*100 + patch (host only). */
+LLMINT8_API int llmint8_version(void);
+
+/*
+ * Offline weight quantisation, once per weight matrix
+ * ('LLM quantization, part 2' §2.1 vector-wise quantization):
+ *   Wscale[n] = max_k |W[n,k]| / 127                       (binary32, IEEE division)
+ *   Wq[n,k]   = clamp(round_half_even(W[n,k] / Wscale[n]), -127, 127), 0 if Wscale[n] == 0
+ * over all K columns.  W: fp16 [N][K] in; Wq: int8 [N][K] out; Wscale: float [N] out.
+ * N >= 1, K >= 16, K % 16 == 0.
+ */
+LLMINT8_API int llmint8_quantize_weight(const void* W, int64_t N, int64_t K, int8_t* Wq, float* Wscale,
+                            void* stream);
+
+/* Bytes of device workspace llmint8_matmul needs for this shape on the AUTO path
+ * (host only; 0 for invalid sizes).  The size covers the worst case |O| = K. */
+LLMINT8_API size_t llmint8_workspace_bytes(int64_t T, int64_t N, int64_t K);
+
+/* Same for an explicit path (LLMINT8_PATH_*); 0 if the path cannot take T. */
+LLMINT8_API size_t llmint8_workspace_bytes_path(int64_t T, int64_t N, int64_t K, int path);
+
+/*
+ * Y = X * W^T by the LLM.int8() decomposition ('LLM quantization, part 2' §2.1;
+ * '三、模型量化' Q4):
+ *   O      = { k : |X[t,k]| >= threshold for some row t of this X }   (ascending)
+ *   sx[t]  = max_{k not in O} |X[t,k]| / 127                           (binary32)
+ *   Xq     = clamp(round_half_even(X / sx), -127, 127) on k not in O, 0 on O
+ *   acc    = Xq * Wq^T                                                 (exact int32)
+ *   yo     = X[:,O] * W[:,O]^T                                         (fp16 in, fp32 sum)
+ *   Y      = fp16( acc * sx[t] * Wscale[n] + yo )
+ * X: fp16 [T][K]; Wq/Wscale from llmint8_quantize_weight(W); W: the fp16 weight
+ * [N][K], read only at the outlier columns; Y: fp16 [T][N] out.
+ * threshold: +inf disables the outlier part; NaN is rejected.
+ * workspace: device scratch of at least llmint8_workspace_bytes(T, N, K) bytes,
+ * owned by the caller, contents on entry ignored; calls that share a workspace
+ * must be ordered on one stream.  The outlier set never returns to the host.
+ * T >= 1, N >= 1, K >= 16, K % 16 == 0, K * 127 * 127 < 2^31.
+ */
+LLMINT8_API int llmint8_matmul(const void* X, int64_t T, int64_t K, const int8_t* Wq, const float* Wscale,
+                   const void* W, int64_t N, float threshold, void* Y, void* workspace,
+                   size_t workspace_bytes, void* stream);
+
+/*
+ * Inspection variant of llmint8_matmul used by the parity tests: `path` picks
+ * the kernel path (LLMINT8_PATH_*); when `acc_out` (int32 [T][N], device) is
+ * not NULL the exact int32 products acc are written there as well.  The
+ * workspace must hold llmint8_workspace_bytes_path(T, N, K, path) bytes.
+ */
+LLMINT8_API int llmint8_matmul_debug(const void* X, int64_t T, int64_t K, const int8_t* Wq,
+                         const float* Wscale, const void* W, int64_t N, float threshold, void* Y,
+                         void* workspace, size_t workspace_bytes, int path, int32_t* acc_out,
+                         void* stream);
+
+/*
+ * Profiling variant of llmint8_matmul_debug: records `ev_main_begin` and
+ * `ev_main_end` (cudaEvent_t, created by the caller, may be NULL) on `stream`
+ * right before and right after the launch of the main kernel (the GEMV or the
+ * GEMM), so the caller can time that kernel alone.  The events sit between
+ * the launches, so the main kernel does not overlap its prologue with the
+ * activation stages here as it does inside llmint8_matmul.
+ */
+LLMINT8_API int llmint8_matmul_profile(const void* X, int64_t T, int64_t K, const int8_t* Wq,
+                                       const float* Wscale, const void* W, int64_t N,
+                                       float threshold, void* Y, void* workspace,
+                                       size_t workspace_bytes, int path, void* ev_main_begin,
+                                       void* ev_main_end, void* stream);
+
+/*
+ * The activation stages of llmint8_matmul alone (outlier detection,
+ * compaction, per-row scale, int8 codes), run by the same kernels in the same
+ * launch configuration as `path` uses inside llmint8_matmul:
+ *   Xq int8 [T][K], xscale float [T], outlier_idx int32 [K] (first *n_outliers
+ *   entries valid, ascending), n_outliers int32 [1]; all device, all outputs.
+ * workspace as for llmint8_matmul_debug with the same path.
+ */
+LLMINT8_API int llmint8_detect_quantize(const void* X, int64_t T, int64_t K, float threshold, int8_t* Xq,
+                            float* xscale, int32_t* outlier_idx, int32_t* n_outliers,
+                            void* workspace, size_t workspace_bytes, int path, void* stream);
+
+/*
+ * Waits for `stream`, then reads and clears this device's error word.
+ * Returns LLMINT8_ERR_TIMEOUT if a kernel gave up a bounded wait since the
+ * last call, LLMINT8_ERR_CUDA if the stream reported an error, else OK.
+ */
+LLMINT8_API int llmint8_sync_status(void* stream);
+
+/*
+ * Self-test of the failure path: launches one kernel that waits on an
+ * mbarrier no thread ever arrives at, gives up after `wait_ns` nanoseconds
+ * (1 000 .. 2e9), records LLMINT8_ERR_TIMEOUT in the error word and returns
+ * normally.  A following llmint8_sync_status() must report the timeout.
+ */
+LLMINT8_API int llmint8_selftest_timeout(uint64_t wait_ns, void* stream);
+
+/* Per-wait limit used by every kernel's bounded waits (default 2 s). */
+LLMINT8_API int llmint8_set_wait_limit_ns(uint64_t ns);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* LLMINT8_H */

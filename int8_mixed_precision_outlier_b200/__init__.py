@@ -1,0 +1,12 @@
+"""LLM.int8() mixed-precision decomposition matmul for B200 (sm_100a).
+
+The compute path is the C-ABI library libllmint8.so (include/llmint8.h); the
+functions here are its Python binding.
+"""
+from .llmint8 import (  # noqa: F401
+    GEMV_MAX_T, PATH_AUTO, PATH_GEMM, PATH_GEMV, Int8Linear, LLMInt8Error, alloc_workspace,
+    header_functions, llmint8_detect_quantize, llmint8_matmul, llmint8_matmul_debug, llmint8_matmul_profile,
+    llmint8_quantize_weight, llmint8_selftest_timeout, llmint8_set_wait_limit_ns,
+    llmint8_status_string, llmint8_sync_status, llmint8_version, llmint8_workspace_bytes,
+    load_library,
+)

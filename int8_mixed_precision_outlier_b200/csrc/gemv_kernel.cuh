@@ -1,0 +1,312 @@
+// gemv_kernel.cuh -- decode-shaped LLM.int8() matmul (T <= 16 tokens).
+//
+// The int8 product acc = Xq * Wq^T is bound by reading Wq from HBM (decode
+// reads every weight once per token batch: '三、模型量化' (lowentro.cn) Q15;
+// 'LLM 量化' (llm-inference-handbook), why quantize).  The kernel streams Wq
+// with TMA and multiplies on the tensor cores with the operands swapped:
+// A = a 128-row tile of Wq (MMA M = 128 output channels), B = the int8 codes
+// of the T tokens padded to 16 (MMA N = 16), D = int32 in TMEM.
+//
+// Work split (stream-K): the N/128 x K/128 k-blocks are cut into one
+// contiguous range per CTA, so every CTA streams the same number of weight
+// bytes.  A range may start or end inside a tile; such partial int32 sums go
+// to a per-CTA slot in the workspace and the last CTA to arrive at a tile
+// (per-tile counter, no spinning) adds them -- exact in int32, so the order
+// does not matter -- and runs the epilogue:
+//   Y[t,n] = fp16( acc[t,n] * sx[t] * sw[n] + yo[t,n] ),
+//   yo[t,n] = sum_{j<|O|} X[t,O_j] * W[n,O_j]   (fp32, ascending j)
+// ('LLM quantization, part 2' (hncyxsy.com) §2.1: the outlier columns in
+// fp16, the rest in int8, the two results added).
+//
+// Warp roles: warp 0 lane 0 issues TMA, warp 1 lane 0 issues tcgen05.mma and
+// owns the TMEM allocation, warps 2-5 (128 threads = 128 TMEM lanes) drain the
+// accumulators.  Two 16-column accumulators let the MMA of one segment
+// overlap the epilogue of the previous one.  Every mbarrier wait is bounded.
+#pragma once
+#include <cuda_fp16.h>
+#include "sm100.cuh"
+
+namespace llmint8 {
+namespace gemv {
+
+constexpr int BM = 128;                    // weight rows per tile = MMA M
+constexpr int BK = 128;                    // K bytes per k-block (one 128 B swizzle row)
+constexpr int NT = 16;                     // tokens per MMA (MMA N)
+constexpr int STAGES = 8;
+constexpr int A_BYTES = BM * BK;           // 16 KiB
+constexpr int B_BYTES = NT * BK;           // 2 KiB
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr int THREADS = 192;
+constexpr int TMEM_COLS = 32;              // 2 accumulators x 16 columns
+constexpr int XO_CHUNK = 64;               // outlier columns staged per epilogue pass
+constexpr int MAX_CTAS = 256;              // partial-slot capacity of the workspace
+constexpr int SLOT_INTS = BM * NT;         // one partial tile, int32 [128][16]
+
+// bytes of dynamic shared memory: stages + barriers/bookkeeping + epilogue staging
+constexpr int SMEM_BYTES = 1024 /*align slack*/ + STAGES * STAGE_BYTES + 256 +
+                           NT * XO_CHUNK * 4 + XO_CHUNK * 4;
+
+struct Params {
+  int T, N, K;
+  int KB;         // k-blocks per tile = ceil(K / BK)
+  int num_tiles;  // ceil(N / BM)
+  int units;      // num_tiles * KB
+  int grid;       // CTAs (<= units, <= MAX_CTAS)
+  const float* sx;
+  const float* sw;
+  const uint16_t* X;
+  const uint16_t* W;
+  const int32_t* idx;
+  const int32_t* n_out;
+  int32_t* counters;  // [num_tiles], zeroed by the prep kernel
+  int32_t* partials;  // [grid][2][BM][NT]
+  uint16_t* Y;
+  int32_t* acc_out;   // optional int32 [T][N]
+  uint64_t wait_ns;
+};
+
+__device__ __forceinline__ int unit_begin(int c, const Params& p) {
+  return static_cast<int>((static_cast<int64_t>(c) * p.units) / p.grid);
+}
+
+// CTA whose range holds unit u.
+__device__ __forceinline__ int cta_of_unit(int u, const Params& p) {
+  int c = static_cast<int>((static_cast<int64_t>(u) * p.grid) / p.units);
+  while (c + 1 < p.grid && unit_begin(c + 1, p) <= u) ++c;
+  while (c > 0 && unit_begin(c, p) > u) --c;
+  return c;
+}
+
+__global__ void __launch_bounds__(THREADS, 1)
+    gemv_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_x,
+                const Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
+  uint64_t* empty = full + STAGES;
+  uint64_t* tfull = empty + STAGES;  // [2]
+  uint64_t* tempty = tfull + 2;      // [2]
+  uint64_t* done = tempty + 2;       // [1]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
+  volatile int* last_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  float* xo_s = reinterpret_cast<float*>(smem + STAGES * STAGE_BYTES + 256);  // [NT][XO_CHUNK]
+  int32_t* idx_s = reinterpret_cast<int32_t*>(xo_s + NT * XO_CHUNK);          // [XO_CHUNK]
+
+  const int warp = static_cast<int>(warp_id());
+  const int lane = static_cast<int>(lane_id());
+  const int cta = blockIdx.x;
+  const int u0 = unit_begin(cta, p);
+  const int u1 = unit_begin(cta + 1, p);
+
+  if (warp == 0 && lane == 0) {
+    prefetch_tensormap(&tmap_w);
+    prefetch_tensormap(&tmap_x);
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&tfull[b], 1);
+      mbar_init(&tempty[b], 4);
+    }
+    mbar_init(done, 1);
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  auto stage_a = [&](int s) { return smem + s * STAGE_BYTES; };
+  auto stage_b = [&](int s) { return smem + s * STAGE_BYTES + A_BYTES; };
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      const uint64_t pol = policy_evict_first();
+      const int n_units = u1 - u0;
+      const int pre = n_units < STAGES ? n_units : STAGES;
+      // The weights do not depend on the preceding kernel: start streaming
+      // them before waiting for it.
+      for (int i = 0; i < pre; ++i) {
+        const int u = u0 + i;
+        mbar_arrive_expect_tx(&full[i], STAGE_BYTES);
+        tma_load_2d_hint(stage_a(i), &tmap_w, &full[i], (u % p.KB) * BK, (u / p.KB) * BM, pol);
+      }
+      pdl_wait();
+      for (int i = 0; i < pre; ++i) {
+        const int u = u0 + i;
+        tma_load_2d(stage_b(i), &tmap_x, &full[i], (u % p.KB) * BK, 0);
+      }
+      int issued = pre;
+      bool ok = true;
+      for (int i = pre; i < n_units && ok; ++i) {
+        const int s = i % STAGES;
+        ok = mbar_wait(&empty[s], ((i / STAGES) & 1) ^ 1, p.wait_ns, kErrTimeoutProducer);
+        if (!ok) break;
+        const int u = u0 + i;
+        mbar_arrive_expect_tx(&full[s], STAGE_BYTES);
+        tma_load_2d_hint(stage_a(s), &tmap_w, &full[s], (u % p.KB) * BK, (u / p.KB) * BM, pol);
+        tma_load_2d(stage_b(s), &tmap_x, &full[s], (u % p.KB) * BK, 0);
+        ++issued;
+      }
+      // Leave no copy in flight: wait for the last loads of every stage.
+      for (int i = issued - STAGES < 0 ? 0 : issued - STAGES; i < issued; ++i)
+        mbar_wait(&full[i % STAGES], (i / STAGES) & 1, p.wait_ns, kErrTimeoutProducer);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_i8_s32(BM, NT);
+      int i = 0, seg = 0;
+      bool ok = true;
+      for (int u = u0; u < u1 && ok; ++seg) {
+        const int tile = u / p.KB;
+        const int seg_end = min(u1, (tile + 1) * p.KB);
+        const int buf = seg & 1;
+        if (seg >= 2) {
+          ok = mbar_wait(&tempty[buf], ((seg >> 1) - 1) & 1, p.wait_ns, kErrTimeoutMma);
+          if (!ok) break;
+        }
+        tc_fence_after();
+        const uint32_t d = tmem_base + static_cast<uint32_t>(buf * NT);
+        const int seg_start = u;
+        for (; u < seg_end; ++u, ++i) {
+          const int s = i % STAGES;
+          ok = mbar_wait(&full[s], (i / STAGES) & 1, p.wait_ns, kErrTimeoutMma);
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t a0 = smem_addr(stage_a(s));
+          const uint32_t b0 = smem_addr(stage_b(s));
+#pragma unroll
+          for (int k = 0; k < BK / 32; ++k)
+            mma_i8(d, make_sdesc_k_sw128(a0 + k * 32), make_sdesc_k_sw128(b0 + k * 32), idesc,
+                   (u > seg_start || k > 0) ? 1u : 0u);
+          mma_commit(&empty[s]);
+        }
+        if (ok) mma_commit(&tfull[buf]);
+      }
+      // All issued MMAs complete before TMEM is released.
+      mma_commit(done);
+      mbar_wait(done, 0, p.wait_ns, kErrTimeoutMma);
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    pdl_wait();
+    const int q = warp & 3;                  // TMEM lane quadrant of this warp
+    const int row = q * 32 + lane;           // tile row = TMEM lane
+    const int etid = threadIdx.x - 64;       // 0..127
+    const int nO = *p.n_out;
+    const int T = p.T;
+    int seg = 0;
+    for (int u = u0; u < u1; ++seg) {
+      const int tile = u / p.KB;
+      const int kb_begin = u % p.KB;
+      const int seg_end = min(u1, (tile + 1) * p.KB);
+      const bool whole = (kb_begin == 0) && (seg_end == (tile + 1) * p.KB);
+      u = seg_end;
+      const int buf = seg & 1;
+      // All 128 epilogue threads agree on the outcome before going on, so a
+      // timeout can never leave some of them at a named barrier.
+      const bool ok = mbar_wait(&tfull[buf], (seg >> 1) & 1, p.wait_ns, kErrTimeoutEpilogue);
+      if (!named_barrier_and(2, 128, ok)) break;
+      tc_fence_after();
+      uint32_t r[16];
+      tmem_ld16(tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(buf * NT), r);
+      tmem_ld_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tempty[buf]);
+      int32_t acc[16];
+#pragma unroll
+      for (int t = 0; t < 16; ++t) acc[t] = static_cast<int32_t>(r[t]);
+
+      if (!whole) {
+        const int c_first = cta_of_unit(tile * p.KB, p);
+        const int c_last = cta_of_unit((tile + 1) * p.KB - 1, p);
+        const int slot = (tile == u0 / p.KB) ? 0 : 1;
+        int4* mine = reinterpret_cast<int4*>(p.partials +
+                                             (static_cast<int64_t>(cta) * 2 + slot) * SLOT_INTS + row * NT);
+#pragma unroll
+        for (int v = 0; v < 4; ++v) mine[v] = make_int4(acc[4 * v], acc[4 * v + 1], acc[4 * v + 2], acc[4 * v + 3]);
+        __threadfence();
+        named_barrier(1, 128);
+        if (etid == 0) {
+          const int old = atomicAdd(&p.counters[tile], 1);
+          *last_flag = (old == c_last - c_first) ? 1 : 0;
+        }
+        named_barrier(1, 128);
+        const bool last = *last_flag != 0;
+        if (!last) continue;
+        __threadfence();
+        for (int c2 = c_first; c2 <= c_last; ++c2) {
+          if (c2 == cta) continue;
+          const int slot2 = (tile == unit_begin(c2, p) / p.KB) ? 0 : 1;
+          const int4* other = reinterpret_cast<const int4*>(
+              p.partials + (static_cast<int64_t>(c2) * 2 + slot2) * SLOT_INTS + row * NT);
+#pragma unroll
+          for (int v = 0; v < 4; ++v) {
+            const int4 o = __ldcg(other + v);
+            acc[4 * v] += o.x;
+            acc[4 * v + 1] += o.y;
+            acc[4 * v + 2] += o.z;
+            acc[4 * v + 3] += o.w;
+          }
+        }
+      }
+
+      // ---- finalize this tile: outlier product, dequantisation, fp16 store
+      const int n = tile * BM + row;
+      float yo[16];
+#pragma unroll
+      for (int t = 0; t < 16; ++t) yo[t] = 0.0f;
+      for (int j0 = 0; j0 < nO; j0 += XO_CHUNK) {
+        const int cnt = min(XO_CHUNK, nO - j0);
+        named_barrier(1, 128);
+        for (int e = etid; e < NT * XO_CHUNK; e += 128) {
+          const int t = e / XO_CHUNK, jj = e % XO_CHUNK;
+          float v = 0.0f;
+          if (t < T && jj < cnt) v = half_bits_to_float(p.X[static_cast<int64_t>(t) * p.K + p.idx[j0 + jj]]);
+          xo_s[e] = v;
+        }
+        if (etid < XO_CHUNK) idx_s[etid] = etid < cnt ? p.idx[j0 + etid] : 0;
+        named_barrier(1, 128);
+        if (n < p.N) {
+          const uint16_t* wrow = p.W + static_cast<int64_t>(n) * p.K;
+          for (int jj = 0; jj < cnt; ++jj) {
+            const float w = half_bits_to_float(__ldg(wrow + idx_s[jj]));
+#pragma unroll
+            for (int t = 0; t < 16; ++t) yo[t] = fmaf(xo_s[t * XO_CHUNK + jj], w, yo[t]);
+          }
+        }
+      }
+      if (n < p.N) {
+        const float swn = p.sw[n];
+#pragma unroll
+        for (int t = 0; t < 16; ++t) {
+          if (t < T) {
+            const float y = static_cast<float>(acc[t]) * p.sx[t] * swn + yo[t];
+            p.Y[static_cast<int64_t>(t) * p.N + n] = __half_as_ushort(__float2half_rn(y));
+            if (p.acc_out) p.acc_out[static_cast<int64_t>(t) * p.N + n] = acc[t];
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem_base, TMEM_COLS);
+  }
+}
+
+}  // namespace gemv
+}  // namespace llmint8

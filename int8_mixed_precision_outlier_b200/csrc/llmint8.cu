@@ -1,0 +1,463 @@
+// llmint8.cu -- the C ABI (include/llmint8.h) over the sm_100a kernels.
+//
+// One translation unit: the kernels live in the .cuh files included below so
+// that the per-device error word is a single __device__ symbol without
+// relocatable device code.  Host code here only validates arguments, lays out
+// the caller's workspace, encodes TMA tensor maps and launches; every step of
+// the method runs in the kernels.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "llmint8.h"
+
+#include "gemm_kernel.cuh"
+#include "gemv_kernel.cuh"
+#include "prep_kernels.cuh"
+#include "sm100.cuh"
+
+namespace llmint8 {
+namespace {
+
+constexpr int kVersion = 100;  // 0.1.0
+constexpr int kMaxDevices = 64;
+constexpr int64_t kMaxK = 65536;         // decode prep keeps K/8 mask bytes in shared memory
+constexpr int64_t kMaxInt32Sum = 133143; // K * 127 * 127 < 2^31
+constexpr int kDetectTargetCtas = 592;   // 4 x 148 SMs
+
+std::atomic<uint64_t> g_wait_ns{2000000000ull};
+
+// ------------------------------------------------------------ device facts
+struct DeviceInfo {
+  std::once_flag once;
+  int status = LLMINT8_OK;
+  int num_sms = 0;
+};
+DeviceInfo g_dev[kMaxDevices];
+
+int device_info(int* num_sms) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return LLMINT8_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return LLMINT8_ERR_CUDA;
+  DeviceInfo& d = g_dev[dev];
+  std::call_once(d.once, [&]() {
+    int major = 0, minor = 0, sms = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+      d.status = LLMINT8_ERR_CUDA;
+      return;
+    }
+    if (major != 10 || minor != 0) {
+      d.status = LLMINT8_ERR_UNSUPPORTED_ARCH;
+      return;
+    }
+    if (cudaFuncSetAttribute(gemm::gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             gemm::SMEM_BYTES) != cudaSuccess ||
+        cudaFuncSetAttribute(gemv::gemv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             gemv::SMEM_BYTES) != cudaSuccess) {
+      d.status = LLMINT8_ERR_CUDA;
+      return;
+    }
+    d.num_sms = sms;
+  });
+  if (num_sms) *num_sms = d.num_sms;
+  return d.status;
+}
+
+// ------------------------------------------------------------ tensor maps
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static std::once_flag once;
+  static EncodeTiledFn fn = nullptr;
+  std::call_once(once, []() {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 2-D row-major tensor [outer][inner] of `elem_bytes` elements, rows
+// `row_bytes` apart, read in boxes of box_outer rows x box_inner elements
+// (box_inner * elem_bytes == 128: one swizzle row).
+bool encode_2d(CUtensorMap* map, CUtensorMapDataType dt, const void* base, uint64_t inner,
+               uint64_t outer, uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {inner, outer};
+  const cuuint64_t strides[1] = {row_bytes};
+  const cuuint32_t box[2] = {box_inner, box_outer};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(map, dt, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// ------------------------------------------------------------ workspace layout
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+struct Layout {
+  int path = 0;
+  int Kw = 0, R = 0, rows_per_chunk = 0, ldo = 0, num_tiles = 0;
+  size_t part = 0, flags = 0, idx = 0, n_out = 0, counters = 0, sx = 0, xq = 0, xo = 0, wo = 0,
+         partials = 0, total = 0;
+};
+
+bool make_layout(int64_t T, int64_t N, int64_t K, int path, Layout* L) {
+  if (T < 0 || N < 0 || K < 16 || K % 16 != 0 || K > kMaxK) return false;
+  if (path == LLMINT8_PATH_AUTO) path = T <= LLMINT8_GEMV_MAX_T ? LLMINT8_PATH_GEMV : LLMINT8_PATH_GEMM;
+  if (path == LLMINT8_PATH_GEMV && T > LLMINT8_GEMV_MAX_T) return false;
+  if (path != LLMINT8_PATH_GEMV && path != LLMINT8_PATH_GEMM) return false;
+  L->path = path;
+  L->Kw = static_cast<int>((K + 31) / 32);
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = off;
+    off = align_up(off + (bytes ? bytes : 1), 256);
+    return at;
+  };
+  if (path == LLMINT8_PATH_GEMV) {
+    L->num_tiles = static_cast<int>((N + gemv::BM - 1) / gemv::BM);
+    L->flags = take(sizeof(uint32_t) * L->Kw);
+    L->idx = take(sizeof(int32_t) * K);
+    L->n_out = take(sizeof(int32_t));
+    L->counters = take(sizeof(int32_t) * (L->num_tiles ? L->num_tiles : 1));
+    L->sx = take(sizeof(float) * LLMINT8_GEMV_MAX_T);
+    L->xq = take(static_cast<size_t>(LLMINT8_GEMV_MAX_T) * K);
+    L->partials = take(sizeof(int32_t) * gemv::MAX_CTAS * 2 * gemv::SLOT_INTS);
+  } else {
+    const int64_t strips = (K + kDetectCols - 1) / kDetectCols;
+    int64_t R = (kDetectTargetCtas + strips - 1) / strips;
+    const int64_t rmax = T > 0 ? (T + 3) / 4 : 1;
+    if (R > rmax) R = rmax;
+    if (R < 1) R = 1;
+    const int64_t rpc = T > 0 ? (T + R - 1) / R : 1;
+    R = T > 0 ? (T + rpc - 1) / rpc : 1;
+    L->R = static_cast<int>(R);
+    L->rows_per_chunk = static_cast<int>(rpc);
+    L->ldo = static_cast<int>((K + 63) / 64 * 64);
+    L->part = take(sizeof(uint32_t) * static_cast<size_t>(R) * L->Kw);
+    L->flags = take(sizeof(uint32_t) * L->Kw);
+    L->idx = take(sizeof(int32_t) * K);
+    L->n_out = take(sizeof(int32_t));
+    L->sx = take(sizeof(float) * static_cast<size_t>(T));
+    L->xq = take(static_cast<size_t>(T) * K);
+    L->xo = take(sizeof(uint16_t) * static_cast<size_t>(T) * L->ldo);
+    L->wo = take(sizeof(uint16_t) * static_cast<size_t>(N) * L->ldo);
+  }
+  L->total = off;
+  return true;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// ------------------------------------------------------------ launches
+template <typename... Exp, typename... Act>
+cudaError_t launch(void (*kern)(Exp...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, bool pdl,
+                   Act&&... args) {
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg;
+  std::memset(&cfg, 0, sizeof(cfg));
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cfg.attrs = pdl ? attr : nullptr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<Act>(args)...);
+}
+
+struct Prep {
+  // outputs of the activation stages (workspace or caller buffers)
+  int8_t* xq;
+  float* sx;
+  int32_t* idx;
+  int32_t* n_out;
+};
+
+// Activation stages.  GEMV path: one decode prep kernel.  GEMM path: detect,
+// compact, quantize+gather (the W gather only when W != nullptr).
+int launch_prep(const Layout& L, const uint16_t* X, int T, int K, const uint16_t* W, int N, float tau,
+                uint8_t* ws, const Prep& out, cudaStream_t st) {
+  uint32_t* flags = reinterpret_cast<uint32_t*>(ws + L.flags);
+  cudaError_t e;
+  if (L.path == LLMINT8_PATH_GEMV) {
+    int32_t* counters = reinterpret_cast<int32_t*>(ws + L.counters);
+    e = launch(decode_prep_kernel, dim3(1), dim3(kDecodePrepThreads), static_cast<size_t>(K / 8), st,
+               false, X, T, K, tau, flags, out.idx, out.n_out, out.xq, out.sx, counters,
+               W ? L.num_tiles : 0);
+    return e == cudaSuccess ? LLMINT8_OK : LLMINT8_ERR_CUDA;
+  }
+  uint32_t* part = reinterpret_cast<uint32_t*>(ws + L.part);
+  const int strips = (K + kDetectCols - 1) / kDetectCols;
+  e = launch(detect_partial_kernel, dim3(strips, L.R), dim3(kPrepThreads), 0, st, false, X, T, K, tau,
+             L.rows_per_chunk, part, L.Kw);
+  if (e != cudaSuccess) return LLMINT8_ERR_CUDA;
+  e = launch(compact_kernel, dim3(1), dim3(kCompactThreads), 0, st, true,
+             static_cast<const uint32_t*>(part), L.R, L.Kw, flags, out.idx, out.n_out);
+  if (e != cudaSuccess) return LLMINT8_ERR_CUDA;
+  const int wblocks = W ? (N + kWoRowsPerCta - 1) / kWoRowsPerCta : 0;
+  e = launch(quant_gather_kernel, dim3(T + wblocks), dim3(kPrepThreads), 0, st, true, X, T, K, W, N,
+             static_cast<const uint32_t*>(flags), static_cast<const int32_t*>(out.idx),
+             static_cast<const int32_t*>(out.n_out), out.xq, out.sx,
+             reinterpret_cast<uint16_t*>(ws + L.xo), reinterpret_cast<uint16_t*>(ws + L.wo), L.ldo);
+  return e == cudaSuccess ? LLMINT8_OK : LLMINT8_ERR_CUDA;
+}
+
+int check_common(const void* X, int64_t T, int64_t K, float threshold, const void* ws, size_t ws_bytes,
+                 int path, Layout* L, int64_t N) {
+  if (T < 0 || N < 0 || K < 16 || K > kMaxK || K > kMaxInt32Sum) return LLMINT8_ERR_INVALID_ARG;
+  if (T > INT32_MAX || N > INT32_MAX) return LLMINT8_ERR_INVALID_ARG;
+  if (std::isnan(threshold)) return LLMINT8_ERR_INVALID_ARG;
+  if (path < LLMINT8_PATH_AUTO || path > LLMINT8_PATH_GEMM) return LLMINT8_ERR_INVALID_ARG;
+  if (K % 16 != 0) return LLMINT8_ERR_ALIGNMENT;
+  if (!make_layout(T, N, K, path, L)) return LLMINT8_ERR_INVALID_ARG;
+  if (T > 0 && (!X || !ws)) return LLMINT8_ERR_INVALID_ARG;
+  if (T > 0 && (!aligned16(X) || !aligned16(ws))) return LLMINT8_ERR_ALIGNMENT;
+  if (T > 0 && ws_bytes < L->total) return LLMINT8_ERR_WORKSPACE;
+  return LLMINT8_OK;
+}
+
+int matmul_impl(const void* Xv, int64_t T, int64_t K, const int8_t* Wq, const float* Wscale,
+                const void* Wv, int64_t N, float threshold, void* Yv, void* workspace,
+                size_t ws_bytes, int path, int32_t* acc_out, void* stream,
+                cudaEvent_t ev_begin = nullptr, cudaEvent_t ev_end = nullptr) {
+  Layout L;
+  int rc = check_common(Xv, T, K, threshold, workspace, ws_bytes, path, &L, N);
+  if (rc != LLMINT8_OK) return rc;
+  if (T == 0 || N == 0) return LLMINT8_OK;
+  if (!Wq || !Wscale || !Wv || !Yv) return LLMINT8_ERR_INVALID_ARG;
+  if (!aligned16(Wq) || !aligned16(Wv) || !aligned16(Yv) ||
+      (reinterpret_cast<uintptr_t>(Wscale) & 3u) || (reinterpret_cast<uintptr_t>(acc_out) & 3u))
+    return LLMINT8_ERR_ALIGNMENT;
+  int num_sms = 0;
+  rc = device_info(&num_sms);
+  if (rc != LLMINT8_OK) return rc;
+
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const uint16_t* X = static_cast<const uint16_t*>(Xv);
+  const uint16_t* W = static_cast<const uint16_t*>(Wv);
+  uint16_t* Y = static_cast<uint16_t*>(Yv);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  const int t = static_cast<int>(T), n = static_cast<int>(N), k = static_cast<int>(K);
+  Prep out{reinterpret_cast<int8_t*>(ws + L.xq), reinterpret_cast<float*>(ws + L.sx),
+           reinterpret_cast<int32_t*>(ws + L.idx), reinterpret_cast<int32_t*>(ws + L.n_out)};
+  const uint64_t wait_ns = g_wait_ns.load();
+
+  if (L.path == LLMINT8_PATH_GEMV) {
+    gemv::Params p;
+    p.T = t;
+    p.N = n;
+    p.K = k;
+    p.KB = (k + gemv::BK - 1) / gemv::BK;
+    p.num_tiles = L.num_tiles;
+    p.units = p.num_tiles * p.KB;
+    int grid = num_sms < gemv::MAX_CTAS ? num_sms : gemv::MAX_CTAS;
+    if (grid > p.units) grid = p.units;
+    p.grid = grid;
+    p.sx = out.sx;
+    p.sw = Wscale;
+    p.X = X;
+    p.W = W;
+    p.idx = out.idx;
+    p.n_out = out.n_out;
+    p.counters = reinterpret_cast<int32_t*>(ws + L.counters);
+    p.partials = reinterpret_cast<int32_t*>(ws + L.partials);
+    p.Y = Y;
+    p.acc_out = acc_out;
+    p.wait_ns = wait_ns;
+    CUtensorMap tw, tx;
+    if (!encode_2d(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT8, Wq, K, N, K, gemv::BK, gemv::BM) ||
+        !encode_2d(&tx, CU_TENSOR_MAP_DATA_TYPE_UINT8, out.xq, K, T, K, gemv::BK, gemv::NT))
+      return LLMINT8_ERR_CUDA;
+    rc = launch_prep(L, X, t, k, W, n, threshold, ws, out, st);
+    if (rc != LLMINT8_OK) return rc;
+    if (ev_begin && cudaEventRecord(ev_begin, st) != cudaSuccess) return LLMINT8_ERR_CUDA;
+    cudaError_t e = launch(gemv::gemv_kernel, dim3(grid), dim3(gemv::THREADS), gemv::SMEM_BYTES, st, true,
+                           tw, tx, p);
+    if (e != cudaSuccess) return LLMINT8_ERR_CUDA;
+    if (ev_end && cudaEventRecord(ev_end, st) != cudaSuccess) return LLMINT8_ERR_CUDA;
+    return LLMINT8_OK;
+  }
+
+  gemm::Params p;
+  p.T = t;
+  p.N = n;
+  p.K = k;
+  p.KB = (k + gemm::BK - 1) / gemm::BK;
+  p.num_m = (t + gemm::BM - 1) / gemm::BM;
+  p.sx = out.sx;
+  p.sw = Wscale;
+  p.n_out = out.n_out;
+  p.Y = Y;
+  p.acc_out = acc_out;
+  p.wait_ns = wait_ns;
+  const int num_n = (n + gemm::BN - 1) / gemm::BN;
+  CUtensorMap txq, twq, txo, two;
+  const uint16_t* xo = reinterpret_cast<const uint16_t*>(ws + L.xo);
+  const uint16_t* wo = reinterpret_cast<const uint16_t*>(ws + L.wo);
+  if (!encode_2d(&txq, CU_TENSOR_MAP_DATA_TYPE_UINT8, out.xq, K, T, K, gemm::BK, gemm::BM) ||
+      !encode_2d(&twq, CU_TENSOR_MAP_DATA_TYPE_UINT8, Wq, K, N, K, gemm::BK, gemm::BN) ||
+      !encode_2d(&txo, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, xo, L.ldo, T, 2ull * L.ldo, 64, gemm::BM) ||
+      !encode_2d(&two, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, wo, L.ldo, N, 2ull * L.ldo, 64, gemm::BN))
+    return LLMINT8_ERR_CUDA;
+  rc = launch_prep(L, X, t, k, W, n, threshold, ws, out, st);
+  if (rc != LLMINT8_OK) return rc;
+  if (ev_begin && cudaEventRecord(ev_begin, st) != cudaSuccess) return LLMINT8_ERR_CUDA;
+  cudaError_t e = launch(gemm::gemm_kernel, dim3(p.num_m * num_n), dim3(gemm::THREADS), gemm::SMEM_BYTES,
+                         st, true, txq, twq, txo, two, p);
+  if (e != cudaSuccess) return LLMINT8_ERR_CUDA;
+  if (ev_end && cudaEventRecord(ev_end, st) != cudaSuccess) return LLMINT8_ERR_CUDA;
+  return LLMINT8_OK;
+}
+
+__global__ void selftest_timeout_kernel(uint64_t wait_ns) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_barrier_init();
+  }
+  __syncthreads();
+  // Phase 0 of `bar` never completes: nothing arrives on it.
+  if (threadIdx.x == 0) mbar_wait(&bar, 0, wait_ns, kErrTimeoutSelftest);
+  __syncthreads();
+}
+
+}  // namespace
+}  // namespace llmint8
+
+using namespace llmint8;
+
+extern "C" {
+
+const char* llmint8_status_string(int status) {
+  switch (status) {
+    case LLMINT8_OK: return "ok";
+    case LLMINT8_ERR_INVALID_ARG: return "invalid argument";
+    case LLMINT8_ERR_ALIGNMENT: return "misaligned pointer or K not a multiple of 16";
+    case LLMINT8_ERR_UNSUPPORTED_ARCH: return "device is not sm_100 (B200)";
+    case LLMINT8_ERR_WORKSPACE: return "workspace too small";
+    case LLMINT8_ERR_CUDA: return "CUDA runtime error";
+    case LLMINT8_ERR_TIMEOUT: return "a kernel gave up a bounded wait";
+    case LLMINT8_ERR_UNIMPLEMENTED: return "not implemented";
+    default: return "unknown status";
+  }
+}
+
+int llmint8_version(void) { return kVersion; }
+
+int llmint8_set_wait_limit_ns(uint64_t ns) {
+  if (ns < 1000ull || ns > 60000000000ull) return LLMINT8_ERR_INVALID_ARG;
+  g_wait_ns.store(ns);
+  return LLMINT8_OK;
+}
+
+size_t llmint8_workspace_bytes_path(int64_t T, int64_t N, int64_t K, int path) {
+  Layout L;
+  if (N < 0 || K > kMaxInt32Sum || !make_layout(T, N, K, path, &L)) return 0;
+  return L.total;
+}
+
+size_t llmint8_workspace_bytes(int64_t T, int64_t N, int64_t K) {
+  return llmint8_workspace_bytes_path(T, N, K, LLMINT8_PATH_AUTO);
+}
+
+int llmint8_quantize_weight(const void* W, int64_t N, int64_t K, int8_t* Wq, float* Wscale, void* stream) {
+  if (N < 0 || N > INT32_MAX || K < 16 || K > kMaxInt32Sum) return LLMINT8_ERR_INVALID_ARG;
+  if (K % 16 != 0) return LLMINT8_ERR_ALIGNMENT;
+  if (N == 0) return LLMINT8_OK;
+  if (!W || !Wq || !Wscale) return LLMINT8_ERR_INVALID_ARG;
+  if (!aligned16(W) || !aligned16(Wq) || (reinterpret_cast<uintptr_t>(Wscale) & 3u))
+    return LLMINT8_ERR_ALIGNMENT;
+  int rc = device_info(nullptr);
+  if (rc != LLMINT8_OK) return rc;
+  cudaError_t e = launch(quantize_weight_kernel, dim3(static_cast<unsigned>(N)), dim3(kPrepThreads), 0,
+                         static_cast<cudaStream_t>(stream), false, static_cast<const uint16_t*>(W),
+                         static_cast<int>(K), Wq, Wscale);
+  return e == cudaSuccess ? LLMINT8_OK : LLMINT8_ERR_CUDA;
+}
+
+int llmint8_matmul(const void* X, int64_t T, int64_t K, const int8_t* Wq, const float* Wscale,
+                   const void* W, int64_t N, float threshold, void* Y, void* workspace,
+                   size_t workspace_bytes, void* stream) {
+  return matmul_impl(X, T, K, Wq, Wscale, W, N, threshold, Y, workspace, workspace_bytes,
+                     LLMINT8_PATH_AUTO, nullptr, stream);
+}
+
+int llmint8_matmul_debug(const void* X, int64_t T, int64_t K, const int8_t* Wq, const float* Wscale,
+                         const void* W, int64_t N, float threshold, void* Y, void* workspace,
+                         size_t workspace_bytes, int path, int32_t* acc_out, void* stream) {
+  return matmul_impl(X, T, K, Wq, Wscale, W, N, threshold, Y, workspace, workspace_bytes, path,
+                     acc_out, stream);
+}
+
+int llmint8_matmul_profile(const void* X, int64_t T, int64_t K, const int8_t* Wq, const float* Wscale,
+                           const void* W, int64_t N, float threshold, void* Y, void* workspace,
+                           size_t workspace_bytes, int path, void* ev_main_begin, void* ev_main_end,
+                           void* stream) {
+  return matmul_impl(X, T, K, Wq, Wscale, W, N, threshold, Y, workspace, workspace_bytes, path, nullptr,
+                     stream, static_cast<cudaEvent_t>(ev_main_begin), static_cast<cudaEvent_t>(ev_main_end));
+}
+
+int llmint8_detect_quantize(const void* X, int64_t T, int64_t K, float threshold, int8_t* Xq,
+                            float* xscale, int32_t* outlier_idx, int32_t* n_outliers, void* workspace,
+                            size_t workspace_bytes, int path, void* stream) {
+  Layout L;
+  int rc = check_common(X, T, K, threshold, workspace, workspace_bytes, path, &L, 0);
+  if (rc != LLMINT8_OK) return rc;
+  if (!outlier_idx || !n_outliers) return LLMINT8_ERR_INVALID_ARG;
+  if (T > 0 && (!Xq || !xscale)) return LLMINT8_ERR_INVALID_ARG;
+  if ((T > 0 && !aligned16(Xq)) || (reinterpret_cast<uintptr_t>(xscale) & 3u) ||
+      (reinterpret_cast<uintptr_t>(outlier_idx) & 3u) || (reinterpret_cast<uintptr_t>(n_outliers) & 3u))
+    return LLMINT8_ERR_ALIGNMENT;
+  rc = device_info(nullptr);
+  if (rc != LLMINT8_OK) return rc;
+  if (T == 0) return LLMINT8_OK;
+  Prep out{Xq, xscale, outlier_idx, n_outliers};
+  return launch_prep(L, static_cast<const uint16_t*>(X), static_cast<int>(T), static_cast<int>(K), nullptr,
+                     0, threshold, static_cast<uint8_t*>(workspace), out, static_cast<cudaStream_t>(stream));
+}
+
+int llmint8_sync_status(void* stream) {
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(st) != cudaSuccess) return LLMINT8_ERR_CUDA;
+  uint32_t word = 0;
+  if (cudaMemcpyFromSymbolAsync(&word, g_error_word, sizeof(word), 0, cudaMemcpyDeviceToHost, st) !=
+          cudaSuccess ||
+      cudaStreamSynchronize(st) != cudaSuccess)
+    return LLMINT8_ERR_CUDA;
+  if (word != 0) {
+    const uint32_t zero = 0;
+    if (cudaMemcpyToSymbolAsync(g_error_word, &zero, sizeof(zero), 0, cudaMemcpyHostToDevice, st) !=
+            cudaSuccess ||
+        cudaStreamSynchronize(st) != cudaSuccess)
+      return LLMINT8_ERR_CUDA;
+    return LLMINT8_ERR_TIMEOUT;
+  }
+  return LLMINT8_OK;
+}
+
+int llmint8_selftest_timeout(uint64_t wait_ns, void* stream) {
+  if (wait_ns < 1000ull || wait_ns > 2000000000ull) return LLMINT8_ERR_INVALID_ARG;
+  int rc = device_info(nullptr);
+  if (rc != LLMINT8_OK) return rc;
+  cudaError_t e = launch(selftest_timeout_kernel, dim3(1), dim3(32), 0, static_cast<cudaStream_t>(stream),
+                         false, wait_ns);
+  return e == cudaSuccess ? LLMINT8_OK : LLMINT8_ERR_CUDA;
+}
+
+}  // extern "C"

@@ -1,0 +1,114 @@
+"""The C-ABI library without a GPU: it builds, loads, exports every entry point
+include/llmint8.h declares, and rejects bad arguments before any CUDA call.
+
+Only host-side paths run here: argument validation returns before the library
+touches the device, so fake (never dereferenced) pointers are safe.
+"""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+import int8_mixed_precision_outlier_b200 as L
+from int8_mixed_precision_outlier_b200 import _build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    _build.build()
+    return L.load_library()
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = L.header_functions()
+    assert len(names) >= 10
+    for n in names:
+        assert getattr(lib, n) is not None
+    out = subprocess.run(["nm", "-D", "--defined-only", _build.LIB], capture_output=True,
+                         text=True, check=True).stdout
+    exported = set(re.findall(r"\sT\s(llmint8_\w+)", out))
+    assert exported == set(names)
+
+
+def test_status_strings_and_version(lib):
+    assert L.llmint8_version() >= 100
+    for s in range(-7, 1):
+        assert L.llmint8_status_string(s)
+    assert "timeout" in L.llmint8_status_string(-6) or "bounded wait" in L.llmint8_status_string(-6)
+
+
+def test_workspace_sizes(lib):
+    ws = L.llmint8_workspace_bytes
+    assert ws(16, 11008, 4096) == ws(16, 11008, 4096, L.PATH_GEMV)
+    assert ws(17, 11008, 4096) == ws(17, 11008, 4096, L.PATH_GEMM)
+    assert ws(17, 11008, 4096, L.PATH_GEMV) == 0          # decode path takes T <= 16 only
+    assert ws(4, 100, 24) == 0 and ws(4, 100, 8) == 0      # K must be a multiple of 16, >= 16
+    assert ws(4, 100, 65536 + 16) == 0                     # K limit
+    # the prefill workspace holds Xq, the gathered Xo and Wo at worst case |O| = K
+    T, N, K = 2048, 4096, 4096
+    assert ws(T, N, K) >= T * K + 2 * T * K + 2 * N * K
+    assert ws(T, 2 * N, K) > ws(T, N, K)
+
+
+def _fake(addr):
+    return ctypes.c_void_p(addr)
+
+
+def test_validation_before_any_device_call(lib):
+    A = _fake(0x10000)  # aligned, never dereferenced: validation fails first
+    big = 1 << 40
+    # NaN threshold
+    assert lib.llmint8_matmul(A, 4, 64, A, A, A, 8, float("nan"), A, A, big, None) == -1
+    # K not a multiple of 16
+    assert lib.llmint8_matmul(A, 4, 72, A, A, A, 8, 6.0, A, A, big, None) == -2
+    # misaligned X
+    assert lib.llmint8_matmul(_fake(0x10002), 4, 64, A, A, A, 8, 6.0, A, A, big, None) == -2
+    # workspace too small
+    assert lib.llmint8_matmul(A, 4, 64, A, A, A, 8, 6.0, A, A, 16, None) == -4
+    # null workspace / null output
+    assert lib.llmint8_matmul(A, 4, 64, A, A, A, 8, 6.0, A, None, big, None) == -1
+    assert lib.llmint8_matmul(A, 4, 64, A, A, A, 8, 6.0, None, A, big, None) == -1
+    # bad path; decode path with T > 16
+    assert lib.llmint8_matmul_debug(A, 4, 64, A, A, A, 8, 6.0, A, A, big, 7, None, None) == -1
+    assert lib.llmint8_matmul_debug(A, 17, 64, A, A, A, 8, 6.0, A, A, big, 1, None, None) == -1
+    # K so large that an int32 sum could overflow
+    assert lib.llmint8_matmul(A, 4, 140000, A, A, A, 8, 6.0, A, A, big, None) == -1
+    # weight quantisation
+    assert lib.llmint8_quantize_weight(A, 8, 8, A, A, None) == -1
+    assert lib.llmint8_quantize_weight(A, 8, 24, A, A, None) == -2
+    assert lib.llmint8_quantize_weight(None, 8, 64, A, A, None) == -1
+    # empty problems are valid no-ops
+    assert lib.llmint8_matmul(None, 0, 64, A, A, A, 8, 6.0, A, None, 0, None) == 0
+    assert lib.llmint8_matmul(A, 4, 64, A, A, A, 0, 6.0, A, A, big, None) == 0
+    assert lib.llmint8_quantize_weight(A, 0, 64, A, A, None) == 0
+    # wait limit bounds
+    assert lib.llmint8_set_wait_limit_ns(10) == -1
+    assert lib.llmint8_set_wait_limit_ns(2_000_000_000) == 0
+    assert lib.llmint8_selftest_timeout(10, None) == -1
+
+
+def test_missing_library_fails_loudly(tmp_path):
+    from int8_mixed_precision_outlier_b200 import llmint8 as B
+    with pytest.raises(OSError):
+        B._declare  # noqa: B018  (module loads fine without the library)
+        saved = B._LIB
+        try:
+            B._LIB = None
+            B.load_library(str(tmp_path / "nope.so"))
+        finally:
+            B._LIB = saved
+
+
+def test_product_code_never_touches_the_oracle():
+    pkg = os.path.join(ROOT, "int8_mixed_precision_outlier_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h")):
+                src = open(os.path.join(dirpath, f), encoding="utf-8").read()
+                assert not re.search(r"^\s*(from|import)\s+oracle", src, re.M), f
+                assert "llmint8_oracle" not in src, f
+                assert "liboracle" not in src, f

@@ -1,0 +1,292 @@
+"""GPU parity: the CUDA path (through the C ABI) against the CPU oracle.
+
+Integer stages (Wq, Wscale, outlier set, Xq, sx, int32 acc) must match bit for
+bit; Y must satisfy |Y_gpu - Y_oracle| <= 1e-3 max|Y_oracle| + 1 fp16 ulp.
+Small cases compare every element; the full-size workloads compare every
+integer stage in full and Y / acc on sampled rows, computed by the oracle one
+row at a time.
+"""
+import numpy as np
+import pytest
+
+from gpu_helpers import assert_equal, assert_y_close
+from int8_mixed_precision_outlier_b200 import synth
+
+pytestmark = pytest.mark.gpu
+
+torch = pytest.importorskip("torch")
+
+
+@pytest.fixture(scope="module")
+def L():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from int8_mixed_precision_outlier_b200 import _build
+    _build.build()
+    import int8_mixed_precision_outlier_b200 as L
+    L.load_library()
+    return L
+
+
+def dev(a):
+    return torch.from_numpy(np.ascontiguousarray(a)).cuda()
+
+
+def host(t):
+    return t.detach().cpu().numpy()
+
+
+def ok_status(L):
+    assert L.llmint8_sync_status() == 0
+
+
+def run_full(L, oracle, X, W, tau, path):
+    """GPU and oracle on every element; returns nothing, asserts parity."""
+    Wq_o, sw_o = oracle.quantize_weight(W)
+    Y_o, im = oracle.matmul(X, Wq_o, sw_o, W, tau, intermediates=True)
+    Xd, Wd = dev(X), dev(W)
+    Wq, sw = L.llmint8_quantize_weight(Wd)
+    T, N = X.shape[0], W.shape[0]
+    acc = torch.empty((T, N), dtype=torch.int32, device="cuda")
+    Y = L.llmint8_matmul_debug(Xd, Wq, sw, Wd, tau, path=path, acc_out=acc)
+    Xq, sx, idx = L.llmint8_detect_quantize(Xd, tau, path=path)
+    torch.cuda.synchronize()
+    ok_status(L)
+    assert_equal(host(Wq), Wq_o, "Wq")
+    assert_equal(host(sw).view(np.uint32), sw_o.view(np.uint32), "Wscale")
+    assert_equal(host(idx), im["idx"], "outlier idx")
+    assert_equal(host(Xq), im["Xq"], "Xq")
+    assert_equal(host(sx).view(np.uint32), im["sx"].view(np.uint32), "sx")
+    assert_equal(host(acc), im["acc"], "acc")
+    assert_y_close(host(Y), Y_o, "Y")
+
+
+# --------------------------------------------------------------- weights
+
+@pytest.mark.parametrize("N,K", [(1, 16), (3, 48), (256, 256), (301, 1040), (17, 4096)])
+def test_quantize_weight_bitexact(L, oracle, N, K):
+    W = synth.make_weight(N, K, seed=N + K, sigma=0.05)
+    W[0, :3] = np.array([0.0, -0.0, 0.0], np.float16)
+    Wq, sw = L.llmint8_quantize_weight(dev(W))
+    Wq_o, sw_o = oracle.quantize_weight(W)
+    assert_equal(host(Wq), Wq_o, "Wq")
+    assert_equal(host(sw).view(np.uint32), sw_o.view(np.uint32), "Wscale")
+
+
+def test_quantize_weight_worked_example_and_zero_row(L, oracle):
+    from conftest import read_golden
+    g = read_golden("worked_example_quant.txt")
+    row = np.zeros(16, np.float32)
+    row[:6] = [float(s) for s in g["input"]]
+    W = np.stack([row, np.zeros(16, np.float32)]).astype(np.float16)
+    Wq, sw = L.llmint8_quantize_weight(dev(W))
+    assert host(Wq)[0, :6].tolist() == [int(s) for s in g["codes"]]
+    assert host(sw)[1] == 0.0 and not host(Wq)[1].any()
+
+
+# --------------------------------------------------------------- activations
+
+@pytest.mark.parametrize("path,T", [(1, 1), (1, 5), (1, 16), (2, 1), (2, 17), (2, 130), (2, 300)])
+@pytest.mark.parametrize("K", [16, 272, 1040, 4096])
+def test_detect_quantize_bitexact(L, oracle, path, T, K):
+    X, _ = synth.make_activations(T, K, seed=T * 7 + K, n_dims=min(3, K), mag=(6.0, 60.0),
+                                  spike_rate=2e-3)
+    for tau in (6.0, float("inf"), 0.0, 2.5):
+        Xq, sx, idx = L.llmint8_detect_quantize(dev(X), tau, path=path)
+        flag = oracle.detect_outliers(X, tau)
+        Xq_o, sx_o = oracle.quantize_activations(X, flag)
+        assert_equal(host(idx), oracle.compact(flag), f"idx tau={tau}")
+        assert_equal(host(Xq), Xq_o, f"Xq tau={tau}")
+        assert_equal(host(sx).view(np.uint32), sx_o.view(np.uint32), f"sx tau={tau}")
+    ok_status(L)
+
+
+@pytest.mark.parametrize("path", [1, 2])
+def test_detect_edge_values(L, oracle, path):
+    K = 64
+    X = np.zeros((4, K), np.float16)
+    X[0, 3] = 6.0                          # exactly the threshold: an outlier
+    X[1, 5] = np.nextafter(np.float16(6.0), np.float16(0))  # just below: not
+    X[2, 9] = -6.0
+    X[2, 10] = 1.5
+    X[3, :] = 0.0                          # zero row: scale 0, codes 0
+    Xq, sx, idx = L.llmint8_detect_quantize(dev(X), 6.0, path=path)
+    assert host(idx).tolist() == [3, 9]
+    flag = oracle.detect_outliers(X, 6.0)
+    Xq_o, sx_o = oracle.quantize_activations(X, flag)
+    assert_equal(host(Xq), Xq_o, "Xq")
+    assert_equal(host(sx).view(np.uint32), sx_o.view(np.uint32), "sx")
+    assert host(sx)[3] == 0.0
+
+
+# --------------------------------------------------------------- the matmul
+
+SMALL = [
+    # (path, T, N, K)
+    (1, 1, 128, 256), (1, 3, 300, 272), (1, 16, 1000, 1024), (1, 7, 129, 16), (1, 16, 256, 4096),
+    (2, 1, 256, 256), (2, 17, 300, 272), (2, 129, 513, 1040), (2, 256, 256, 128),
+    (2, 300, 1000, 1024), (2, 16, 256, 16),
+]
+
+
+@pytest.mark.parametrize("path,T,N,K", SMALL)
+@pytest.mark.parametrize("tau", [6.0, float("inf"), 0.0])
+def test_matmul_small(L, oracle, path, T, N, K, tau):
+    X, W = synth.random_case(T, K, N, seed=T + N + K, n_dims=min(5, K), mag=(6.0, 50.0))
+    run_full(L, oracle, X, W, tau, path)
+
+
+@pytest.mark.parametrize("path", [1, 2])
+def test_tiny_config(L, oracle, path):
+    w = synth.workload("tiny")
+    run_full(L, oracle, w["X"], w["W"], 6.0, path)
+    Xq, sx, idx = L.llmint8_detect_quantize(dev(w["X"]), 6.0, path=path)
+    assert host(idx).tolist() == [7, 100]
+
+
+def test_decode_7b_full(L, oracle):
+    w = synth.workload("7b_decode")
+    X16, W = w["X"], w["W"]
+    Wq_o, sw_o = oracle.quantize_weight(W)
+    Wd = dev(W)
+    Wq, sw = L.llmint8_quantize_weight(Wd)
+    assert_equal(host(Wq), Wq_o, "Wq")
+    assert_equal(host(sw).view(np.uint32), sw_o.view(np.uint32), "Wscale")
+    ws = L.alloc_workspace(16, W.shape[0], W.shape[1], "cuda")
+    for T in (1, 2, 4, 8, 16):
+        X = np.ascontiguousarray(X16[:T])
+        Y_o, im = oracle.matmul(X, Wq_o, sw_o, W, 6.0, intermediates=True)
+        acc = torch.empty((T, W.shape[0]), dtype=torch.int32, device="cuda")
+        Y = L.llmint8_matmul_debug(dev(X), Wq, sw, Wd, 6.0, workspace=ws, path=0, acc_out=acc)
+        Y2 = L.llmint8_matmul(dev(X), Wq, sw, Wd, 6.0, workspace=ws)
+        torch.cuda.synchronize()
+        assert im["nO"] == 4
+        assert_equal(host(acc), im["acc"], f"acc T={T}")
+        assert_y_close(host(Y), Y_o, f"Y T={T}")
+        assert_equal(host(Y2), host(Y), "debug and plain entry agree")
+    ok_status(L)
+
+
+def sampled_rows(T, seed):
+    rng = np.random.default_rng(seed)
+    rows = {0, T - 1, min(127, T - 1), min(128, T - 1)}
+    rows.update(rng.choice(T, size=min(T, 4), replace=False).tolist())
+    return np.array(sorted(rows))
+
+
+def run_sampled(L, oracle, X, W, taus, seed=0):
+    """Full-size check: every integer stage in full, Y and acc on sampled rows."""
+    T, K = X.shape
+    N = W.shape[0]
+    Wq_o, sw_o = oracle.quantize_weight(W)
+    Xd, Wd = dev(X), dev(W)
+    Wq, sw = L.llmint8_quantize_weight(Wd)
+    assert_equal(host(Wq), Wq_o, "Wq")
+    assert_equal(host(sw).view(np.uint32), sw_o.view(np.uint32), "Wscale")
+    ws = L.alloc_workspace(T, N, K, "cuda")
+    acc = torch.empty((T, N), dtype=torch.int32, device="cuda")
+    rows = sampled_rows(T, seed)
+    for tau in taus:
+        flag = oracle.detect_outliers(X, tau)
+        idx_o = oracle.compact(flag)
+        Xq_o, sx_o = oracle.quantize_activations(X, flag)
+        Xq, sx, idx = L.llmint8_detect_quantize(Xd, tau)
+        assert_equal(host(idx), idx_o, f"idx tau={tau}")
+        assert_equal(host(Xq), Xq_o, f"Xq tau={tau}")
+        assert_equal(host(sx).view(np.uint32), sx_o.view(np.uint32), f"sx tau={tau}")
+        Y = L.llmint8_matmul_debug(Xd, Wq, sw, Wd, tau, workspace=ws, acc_out=acc)
+        torch.cuda.synchronize()
+        ok_status(L)
+        Xs = np.ascontiguousarray(X[rows])
+        acc_o = oracle.int8_gemm(np.ascontiguousarray(Xq_o[rows]), Wq_o)
+        yo_o = oracle.outlier_gemm(Xs, W, idx_o)
+        Y_o = oracle.dequant_combine(acc_o, sx_o[rows], sw_o, yo_o)
+        assert_equal(host(acc[rows]), acc_o, f"acc rows tau={tau}")
+        assert_y_close(host(Y[rows]), Y_o, f"Y rows tau={tau}")
+        # a property at any size: Y is finite and the last row was written
+        assert torch.isfinite(Y).all()
+    return rows
+
+
+def test_prefill_7b(L, oracle):
+    w = synth.workload("7b_prefill")
+    run_sampled(L, oracle, w["X"], w["W"], w["thresholds"], seed=1)
+
+
+def test_upproj_13b(L, oracle):
+    w = synth.workload("13b_up")
+    run_sampled(L, oracle, w["X"], w["W"], w["thresholds"], seed=2)
+
+
+def test_upproj_70b_threshold_sweep(L, oracle):
+    w = synth.workload("70b_up")
+    run_sampled(L, oracle, w["X"], w["W"], w["thresholds"], seed=3)
+
+
+# --------------------------------------------------------------- robustness
+
+def test_workspace_reuse_and_garbage(L, oracle):
+    X, W = synth.random_case(300, 1040, 513, seed=5, n_dims=4)
+    Wq_o, sw_o = oracle.quantize_weight(W)
+    Wd = dev(W)
+    Wq, sw = L.llmint8_quantize_weight(Wd)
+    for path in (1, 2):
+        nbytes = max(L.llmint8_workspace_bytes(300, 513, 1040, 2),
+                     L.llmint8_workspace_bytes(16, 513, 1040, 1))
+        ws = torch.randint(0, 255, (nbytes,), dtype=torch.uint8, device="cuda")
+        for T in (16, 3, 300, 1, 16) if path == 2 else (16, 3, 1, 16):
+            Xt = np.ascontiguousarray(X[:T])
+            Y = L.llmint8_matmul_debug(dev(Xt), Wq, sw, Wd, 6.0, workspace=ws, path=path)
+            Y_o = oracle.matmul(Xt, Wq_o, sw_o, W, 6.0)
+            torch.cuda.synchronize()
+            assert_y_close(host(Y), Y_o, f"path {path} T={T}")
+    ok_status(L)
+
+
+@pytest.mark.parametrize("path", [1, 2])
+def test_output_guard_bands(L, oracle, path):
+    T, N, K = 9, 300, 272
+    X, W = synth.random_case(T, K, N, seed=8)
+    Wd = dev(W)
+    Wq, sw = L.llmint8_quantize_weight(Wd)
+    pad = 4096
+    buf = torch.full((T * N + 2 * pad,), 1234.0, dtype=torch.float16, device="cuda")
+    Y = buf[pad:pad + T * N].view(T, N)
+    L.llmint8_matmul_debug(dev(X), Wq, sw, Wd, 6.0, Y=Y, path=path)
+    torch.cuda.synchronize()
+    assert bool((buf[:pad] == 1234.0).all()) and bool((buf[pad + T * N:] == 1234.0).all())
+    assert_y_close(host(Y), oracle.matmul(X, *oracle.quantize_weight(W), W, 6.0), "Y")
+
+
+def test_timeout_path_reports_and_recovers(L, oracle):
+    assert L.llmint8_sync_status() == 0
+    L.llmint8_selftest_timeout(2_000_000)  # 2 ms: nothing ever arrives on the barrier
+    assert L.llmint8_sync_status() == L.llmint8.LLMINT8_ERR_TIMEOUT
+    assert L.llmint8_sync_status() == 0    # cleared
+    X, W = synth.random_case(16, 256, 256, seed=9)
+    run_full(L, oracle, X, W, 6.0, 1)
+
+
+def test_misaligned_pointer_rejected(L):
+    X = torch.zeros((4, 64 + 8), dtype=torch.float16, device="cuda")
+    W = torch.zeros((8, 64), dtype=torch.float16, device="cuda")
+    Wq, sw = L.llmint8_quantize_weight(W)
+    Xbad = X.view(-1)[1:1 + 4 * 64].view(4, 64)  # 2-byte offset
+    ws = L.alloc_workspace(4, 8, 64, "cuda")
+    with pytest.raises(L.LLMInt8Error) as e:
+        L.llmint8_matmul(Xbad, Wq, sw, W, 6.0, workspace=ws)
+    assert e.value.status == -2
+    with pytest.raises(L.LLMInt8Error) as e:
+        L.llmint8_matmul(X[:, :64].contiguous(), Wq, sw, W, float("nan"), workspace=ws)
+    assert e.value.status == -1
+
+
+def test_int8_linear_wrapper(L, oracle):
+    X, W = synth.random_case(40, 512, 96, seed=10)
+    lin = L.Int8Linear(dev(W))
+    Y = lin(dev(X))
+    Y1 = lin(dev(np.ascontiguousarray(X[:1])))
+    torch.cuda.synchronize()
+    Wq_o, sw_o = oracle.quantize_weight(W)
+    assert_y_close(host(Y), oracle.matmul(X, Wq_o, sw_o, W, 6.0), "Y")
+    assert_y_close(host(Y1), oracle.matmul(np.ascontiguousarray(X[:1]), Wq_o, sw_o, W, 6.0), "Y1")
