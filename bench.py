@@ -40,6 +40,28 @@ FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1
 INT8_PER_BF16 = 2.0  # nominal dense ratio: 4.5 POPS int8 / 2.25 PFLOPS bf16
 THRESHOLD = 6.0
 FLUSH_BYTES = 256 << 20
+
+
+class L2Flush:
+    """Evicts L2 between timed steps: writes a 256 MiB buffer (2x L2), then
+    reads a second one, so L2 ends up holding clean lines of neither the
+    workload nor the flush.  Without the read, the timed kernels would also pay
+    for writing back the flush buffer's dirty lines."""
+
+    def __init__(self, device):
+        import torch
+        self.w = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=device)
+        self.r = torch.zeros(FLUSH_BYTES, dtype=torch.uint8, device=device)
+
+    def zero_(self, gate_us: float = 0.0):
+        import torch
+        self.w.zero_()
+        torch.amax(self.r)
+        if gate_us > 0:
+            # a bounded spin of the GPU (no flag, fixed cycle count): the host
+            # enqueues what follows before the GPU gets to it, so the events
+            # measure GPU time, not host launch latency
+            torch.cuda._sleep(int(gate_us * 2000))
 DECODE_TS = (1, 2, 4, 8, 16)
 
 
@@ -205,6 +227,20 @@ class Workload:
         self.bytes_per_step = sum(c["bytes"] for c in self.calls)
         self.ops_per_step = sum(c["ops"] for c in self.calls)
         self.launches_per_step = sum(2 if c["T"] <= 16 else 4 for c in self.calls)
+        self.graph = None
+
+    def capture(self):
+        """One step as a CUDA graph (the kernels keep their programmatic
+        dependent-launch edges); replaying it costs one host call."""
+        import torch
+        self.step()  # first calls on this device happen outside the capture
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            self.step()
+        torch.cuda.synchronize()
+        self.graph = g
+        return g
 
     def _add(self, w, T, tau, ws, share_w=None):
         import torch
@@ -235,12 +271,12 @@ class Workload:
         return self.ops_per_step * steps / seconds / 1e12
 
 
-def time_steps(wl: Workload, steps: int, warmup: int, world: int, flush, run=None):
+def time_steps(wl: Workload, steps: int, warmup: int, world: int, flush, run=None, gate_us=0.0):
     """Events around each step on the launching stream; L2 flushed before each."""
     import torch
     run = run or wl.step
     for _ in range(warmup):
-        flush.zero_()
+        flush.zero_(gate_us)
         run()
     stream = torch.cuda.current_stream()
     starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
@@ -250,7 +286,7 @@ def time_steps(wl: Workload, steps: int, warmup: int, world: int, flush, run=Non
     sampler = ClockSampler(torch.cuda.current_device())
     with sampler:
         for i in range(steps):
-            flush.zero_()
+            flush.zero_(gate_us)
             starts[i].record(stream)
             run()
             ends[i].record(stream)
@@ -260,22 +296,25 @@ def time_steps(wl: Workload, steps: int, warmup: int, world: int, flush, run=Non
     return total_ms, sampler.summary()
 
 
-def time_main_kernel(wl: Workload, steps: int, flush) -> tuple[float, int]:
-    """Average duration of the main kernel (GEMV or GEMM) per launch, CUDA events."""
+def time_main_kernel(wl: Workload, steps: int, flush, repeat: int = 20) -> tuple[float, int]:
+    """Average duration per launch of the main kernel (GEMV or GEMM): CUDA
+    events around `repeat` back-to-back launches, after a flush and a short
+    GPU-side gate so that the host has queued them all."""
     import torch
     L = wl.L
-    pairs = []
+    runs = []
     for _ in range(steps):
-        flush.zero_()
         for c in wl.calls:
+            flush.zero_(gate_us=300.0)
             b = torch.cuda.Event(enable_timing=True)
             e = torch.cuda.Event(enable_timing=True)
-            L.llmint8_matmul_profile(c["X"], c["Wq"], c["sw"], c["W"], c["tau"], c["ws"], c["Y"], b, e)
-            pairs.append((b, e, c))
+            L.llmint8_matmul_profile(c["X"], c["Wq"], c["sw"], c["W"], c["tau"], c["ws"], c["Y"], b, e,
+                                     repeat=repeat)
+            runs.append((b, e, c))
     torch.cuda.synchronize()
-    total = sum(b.elapsed_time(e) for b, e, _ in pairs)
-    algo = sum(c["bytes"] if wl.unit == "GB/s" else c["ops"] for _, _, c in pairs)
-    return total / len(pairs), algo / len(pairs)
+    total = sum(b.elapsed_time(e) for b, e, _ in runs)
+    algo = sum(c["bytes"] if wl.unit == "GB/s" else c["ops"] for _, _, c in runs)
+    return total / (len(runs) * repeat), algo / len(runs)
 
 
 def main_kernel_name(wl: Workload) -> str:
@@ -393,8 +432,9 @@ def workload_config(name: str) -> dict:
     cfg = synth.WORKLOADS[name]
     d = {"workload": name, "T": list(cfg["T"]) if isinstance(cfg["T"], tuple) else cfg["T"],
          "N": cfg["N"], "K": cfg["K"], "threshold": THRESHOLD if name != "70b_up" else
-         list(cfg["thresholds"]), "l2": "flushed before every step (256 MiB write)",
-         "parallelism": "replicas (one independent problem per GPU)"}
+         list(cfg["thresholds"]), "l2": "flushed before every step (256 MiB write, then 256 MiB read of another buffer)",
+         "parallelism": "replicas (one independent problem per GPU)",
+         "timing": "step replayed as a CUDA graph; e2e uses direct API calls"}
     if name == "7b_decode":
         d["layers_per_step"] = len(DECODE_TS)
     return d
@@ -419,15 +459,16 @@ def run_ours(args):
     import int8_mixed_precision_outlier_b200 as L
     L.load_library()
     peaks = load_peaks()
-    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=device)
+    flush = L2Flush(device)
 
     wl = Workload(args.workload, device, seed=rank)
-    total_ms, clocks = time_steps(wl, args.steps, args.warmup, world, flush)
+    wl.capture()
+    total_ms, clocks = time_steps(wl, args.steps, args.warmup, world, flush, run=wl.graph.replay)
     t_max = reduce_max(total_ms, world)
     units = reduce_sum((wl.bytes_per_step if wl.unit == "GB/s" else wl.ops_per_step) * args.steps, world)
     value = units / (t_max * 1e-3) / (1e9 if wl.unit == "GB/s" else 1e12)
     status = L.llmint8_sync_status()
-    kern_ms, algo = time_main_kernel(wl, max(3, args.steps // 4), flush)
+    kern_ms, algo = time_main_kernel(wl, 10, flush)
     line = {
         "metric": METRIC, "value": round(value, 3), "unit": wl.unit, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(t_max / args.steps, 5),
@@ -451,7 +492,8 @@ def run_ours(args):
             if name == args.workload:
                 continue
             w2 = Workload(name, device, taus=(THRESHOLD,))
-            ms, ck = time_steps(w2, args.also_steps, 3, 1, flush)
+            w2.capture()
+            ms, ck = time_steps(w2, args.also_steps, 3, 1, flush, run=w2.graph.replay)
             km, ka = time_main_kernel(w2, 3, flush)
             also.append({"workload": name, "value": round(w2.metric_value(ms * 1e-3, args.also_steps), 2),
                          "unit": w2.unit, "ms_per_call": round(ms / args.also_steps, 4),

@@ -114,36 +114,44 @@ LLMINT8_API int llmint8_matmul(const void* X, int64_t T, int64_t K, const int8_t
 
 /*
  * Inspection variant of llmint8_matmul used by the parity tests: `path` picks
- * the kernel path (LLMINT8_PATH_*); when `acc_out` (int32 [T][N], device) is
- * not NULL the exact int32 products acc are written there as well.  The
- * workspace must hold llmint8_workspace_bytes_path(T, N, K, path) bytes.
+ * the kernel path (LLMINT8_PATH_*), and each non-NULL output receives an
+ * intermediate of that very call (all device buffers, written in full):
+ *   acc_out         int32 [T][N]  the exact int8 products acc
+ *   xq_out          int8  [T][K]  the activation codes Xq (16-byte aligned)
+ *   xscale_out      float [T]     the per-row scales sx
+ *   outlier_idx_out int32 [K]     the outlier columns, ascending (first *n valid)
+ *   n_outliers_out  int32 [1]     |O|
+ * The workspace must hold llmint8_workspace_bytes_path(T, N, K, path) bytes.
  */
 LLMINT8_API int llmint8_matmul_debug(const void* X, int64_t T, int64_t K, const int8_t* Wq,
                          const float* Wscale, const void* W, int64_t N, float threshold, void* Y,
                          void* workspace, size_t workspace_bytes, int path, int32_t* acc_out,
-                         void* stream);
+                         int8_t* xq_out, float* xscale_out, int32_t* outlier_idx_out,
+                         int32_t* n_outliers_out, void* stream);
 
 /*
- * Profiling variant of llmint8_matmul_debug: records `ev_main_begin` and
- * `ev_main_end` (cudaEvent_t, created by the caller, may be NULL) on `stream`
- * right before and right after the launch of the main kernel (the GEMV or the
- * GEMM), so the caller can time that kernel alone.  The events sit between
- * the launches, so the main kernel does not overlap its prologue with the
- * activation stages here as it does inside llmint8_matmul.
+ * Profiling variant of llmint8_matmul_debug: runs the activation stages once,
+ * records `ev_main_begin` (cudaEvent_t, created by the caller), launches the
+ * main kernel (the GEMV or the GEMM) `repeat` times back to back (1..1000;
+ * each launch recomputes the same Y from the same workspace), then records
+ * `ev_main_end`.  (elapsed time) / repeat is the main kernel's duration per
+ * launch as consecutive layers would run it, with the events' own overhead
+ * spread over the repeats.
  */
 LLMINT8_API int llmint8_matmul_profile(const void* X, int64_t T, int64_t K, const int8_t* Wq,
                                        const float* Wscale, const void* W, int64_t N,
                                        float threshold, void* Y, void* workspace,
-                                       size_t workspace_bytes, int path, void* ev_main_begin,
-                                       void* ev_main_end, void* stream);
+                                       size_t workspace_bytes, int path, int repeat,
+                                       void* ev_main_begin, void* ev_main_end, void* stream);
 
 /*
- * The activation stages of llmint8_matmul alone (outlier detection,
- * compaction, per-row scale, int8 codes), run by the same kernels in the same
- * launch configuration as `path` uses inside llmint8_matmul:
+ * The activation stages alone (outlier detection, compaction, per-row scale,
+ * int8 codes), run by the kernels and launch configuration that `path` uses
+ * inside llmint8_matmul (AUTO: the decode kernel for T <= 16, else the
+ * prefill kernels; GEMM: the prefill kernels for any T >= 1):
  *   Xq int8 [T][K], xscale float [T], outlier_idx int32 [K] (first *n_outliers
  *   entries valid, ascending), n_outliers int32 [1]; all device, all outputs.
- * workspace as for llmint8_matmul_debug with the same path.
+ * workspace: llmint8_workspace_bytes_path(T, 0, K, path) bytes.
  */
 LLMINT8_API int llmint8_detect_quantize(const void* X, int64_t T, int64_t K, float threshold, int8_t* Xq,
                             float* xscale, int32_t* outlier_idx, int32_t* n_outliers,

@@ -76,6 +76,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     mbar_init(done, 1);
     fence_barrier_init();
   }
+  __syncwarp();  // warp 0 converged: the CTA barrier counts each warp once
   if (warp == 1) {
     tmem_alloc(tmem_slot, TMEM_COLS);
     tmem_relinquish();
@@ -84,6 +85,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  pdl_launch_dependents();  // the next call's kernels may launch and prefetch
 
   auto stage_a = [&](int s) { return smem + s * STAGE_BYTES; };
   auto stage_b = [&](int s) { return smem + s * STAGE_BYTES + A_BYTES; };
@@ -215,10 +217,13 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
   }
 
+  // Lane 0 of warps 0 and 1 ran a role loop alone: bring each warp back
+  // together first, so the CTA barrier waits for every warp (an aligned
+  // barrier reached twice by one diverged warp would count it twice).
+  __syncwarp();
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
-    __syncwarp();
     tc_fence_after();
     tmem_dealloc(tmem_base, TMEM_COLS);
   }

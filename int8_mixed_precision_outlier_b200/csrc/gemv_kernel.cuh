@@ -1,27 +1,32 @@
 // gemv_kernel.cuh -- decode-shaped LLM.int8() matmul (T <= 16 tokens).
 //
-// The int8 product acc = Xq * Wq^T is bound by reading Wq from HBM (decode
-// reads every weight once per token batch: '三、模型量化' (lowentro.cn) Q15;
-// 'LLM 量化' (llm-inference-handbook), why quantize).  The kernel streams Wq
-// with TMA and multiplies on the tensor cores with the operands swapped:
-// A = a 128-row tile of Wq (MMA M = 128 output channels), B = the int8 codes
-// of the T tokens padded to 16 (MMA N = 16), D = int32 in TMEM.
+// The int8 product acc = Xq * Wq^T is bound by reading Wq from HBM: decode
+// reads every weight once per token batch ('三、模型量化' (lowentro.cn) Q15;
+// 'LLM 量化' (llm-inference-handbook), why quantize).  So the kernel streams Wq
+// with TMA, one 128 x 128-byte tile per stage, and multiplies on the tensor
+// cores with the operands swapped: A = the Wq tile (MMA M = 128 output
+// channels), B = the int8 codes of the T tokens padded to 16 (MMA N = 16),
+// D = int32 in TMEM.  The codes, scales and outlier list come from
+// decode_prep_kernel, which runs while this kernel already streams weights
+// (programmatic dependent launch).
 //
 // Work split (stream-K): the N/128 x K/128 k-blocks are cut into one
 // contiguous range per CTA, so every CTA streams the same number of weight
-// bytes.  A range may start or end inside a tile; such partial int32 sums go
-// to a per-CTA slot in the workspace and the last CTA to arrive at a tile
-// (per-tile counter, no spinning) adds them -- exact in int32, so the order
-// does not matter -- and runs the epilogue:
+// bytes.  A range may start or end inside a tile; such partial int32 sums go to
+// a per-CTA slot in the workspace and the last CTA to arrive at a tile (per-tile
+// counter, no spinning) adds them -- exact in int32, so the order does not
+// matter -- and writes
 //   Y[t,n] = fp16( acc[t,n] * sx[t] * sw[n] + yo[t,n] ),
 //   yo[t,n] = sum_{j<|O|} X[t,O_j] * W[n,O_j]   (fp32, ascending j)
-// ('LLM quantization, part 2' (hncyxsy.com) §2.1: the outlier columns in
-// fp16, the rest in int8, the two results added).
+// ('LLM quantization, part 2' (hncyxsy.com) §2.1: outlier columns in fp16,
+// the rest in int8, the two results added; '三、模型量化' Q2: r' = s * q on
+// each operand).
 //
-// Warp roles: warp 0 lane 0 issues TMA, warp 1 lane 0 issues tcgen05.mma and
-// owns the TMEM allocation, warps 2-5 (128 threads = 128 TMEM lanes) drain the
-// accumulators.  Two 16-column accumulators let the MMA of one segment
-// overlap the epilogue of the previous one.  Every mbarrier wait is bounded.
+// Warp roles (192 threads): warp 0 lane 0 issues TMA; warp 1 lane 0 issues
+// tcgen05.mma and owns TMEM; warps 2-5 (128 threads = 128 TMEM lanes) compute
+// the outlier products while the weights stream, then drain the accumulators.
+// Two 16-column accumulators let the MMA of one segment overlap the epilogue
+// of the previous one.  Every mbarrier wait is bounded.
 #pragma once
 #include <cuda_fp16.h>
 #include "sm100.cuh"
@@ -33,32 +38,30 @@ constexpr int BM = 128;                    // weight rows per tile = MMA M
 constexpr int BK = 128;                    // K bytes per k-block (one 128 B swizzle row)
 constexpr int NT = 16;                     // tokens per MMA (MMA N)
 constexpr int STAGES = 8;
-constexpr int A_BYTES = BM * BK;           // 16 KiB
-constexpr int B_BYTES = NT * BK;           // 2 KiB
+constexpr int A_BYTES = BM * BK;           // 16 KiB of Wq
+constexpr int B_BYTES = NT * BK;           // 2 KiB of activation codes
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr int THREADS = 192;
 constexpr int TMEM_COLS = 32;              // 2 accumulators x 16 columns
 constexpr int XO_CHUNK = 64;               // outlier columns staged per epilogue pass
 constexpr int MAX_CTAS = 256;              // partial-slot capacity of the workspace
 constexpr int SLOT_INTS = BM * NT;         // one partial tile, int32 [128][16]
-
-// bytes of dynamic shared memory: stages + barriers/bookkeeping + epilogue staging
-constexpr int SMEM_BYTES = 1024 /*align slack*/ + STAGES * STAGE_BYTES + 256 +
+constexpr int SMEM_BYTES = 1024 /*alignment slack*/ + STAGES * STAGE_BYTES + 256 +
                            NT * XO_CHUNK * 4 + XO_CHUNK * 4;
 
 struct Params {
   int T, N, K;
-  int KB;         // k-blocks per tile = ceil(K / BK)
-  int num_tiles;  // ceil(N / BM)
-  int units;      // num_tiles * KB
-  int grid;       // CTAs (<= units, <= MAX_CTAS)
+  int KB;             // k-blocks per tile = ceil(K / BK)
+  int num_tiles;      // ceil(N / BM)
+  int units;          // num_tiles * KB
+  int grid;           // CTAs (<= units, <= MAX_CTAS)
   const float* sx;
   const float* sw;
   const uint16_t* X;
   const uint16_t* W;
   const int32_t* idx;
   const int32_t* n_out;
-  int32_t* counters;  // [num_tiles], zeroed by the prep kernel
+  int32_t* counters;  // [num_tiles]: zeroed by the prep kernel, reset by each tile's last CTA
   int32_t* partials;  // [grid][2][BM][NT]
   uint16_t* Y;
   int32_t* acc_out;   // optional int32 [T][N]
@@ -77,9 +80,59 @@ __device__ __forceinline__ int cta_of_unit(int u, const Params& p) {
   return c;
 }
 
+// yo[t] = sum_{j<|O|} X[t, O_j] * W[n, O_j] (fp32, ascending j) for the tile row
+// n = tile * BM + row, t < TMAX (zero past T).  All 128 epilogue threads call
+// this together: they stage X's outlier values of 64 columns at a time in
+// shared memory, then each thread gathers its row's weights 8 at a time so
+// that the loads are in flight together.
+template <int TMAX>
+__device__ __forceinline__ void outlier_product(const Params& p, int nO, int tile, int row, int etid,
+                                                float* xo_s, int32_t* idx_s, float (&yo)[TMAX]) {
+#pragma unroll
+  for (int t = 0; t < TMAX; ++t) yo[t] = 0.0f;
+  const int n = tile * BM + row;
+  for (int j0 = 0; j0 < nO; j0 += XO_CHUNK) {
+    const int cnt = min(XO_CHUNK, nO - j0);
+    named_barrier(1, 128);  // the previous chunk has been read
+    if (etid < XO_CHUNK) idx_s[etid] = etid < cnt ? p.idx[j0 + etid] : 0;
+    named_barrier(1, 128);
+    constexpr int PER = (TMAX * XO_CHUNK + 127) / 128;
+    float v[PER];
+#pragma unroll
+    for (int i = 0; i < PER; ++i) {
+      const int e = etid + 128 * i;
+      const int t = e / XO_CHUNK, jj = e % XO_CHUNK;
+      v[i] = (t < p.T && jj < cnt)
+                 ? half_bits_to_float(p.X[static_cast<int64_t>(t) * p.K + idx_s[jj]])
+                 : 0.0f;
+    }
+#pragma unroll
+    for (int i = 0; i < PER; ++i)
+      if (etid + 128 * i < TMAX * XO_CHUNK) xo_s[etid + 128 * i] = v[i];
+    named_barrier(1, 128);
+    if (n < p.N) {
+      const uint16_t* wrow = p.W + static_cast<int64_t>(n) * p.K;
+      for (int jj0 = 0; jj0 < cnt; jj0 += 8) {
+        float w[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+          w[u] = (jj0 + u < cnt) ? half_bits_to_float(__ldg(wrow + idx_s[jj0 + u])) : 0.0f;
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+#pragma unroll
+          for (int t = 0; t < TMAX; ++t) yo[t] = fmaf(xo_s[t * XO_CHUNK + jj0 + u], w[u], yo[t]);
+      }
+    }
+  }
+}
+
+// TMAX: T rounded up to a power of two (1, 2, 4, 8 or 16); the per-token
+// registers and loops of the epilogue are sized by it.
+template <int TMAX>
 __global__ void __launch_bounds__(THREADS, 1)
     gemv_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_x,
                 const Params p) {
+  static_assert(TMAX >= 1 && TMAX <= NT && (TMAX & (TMAX - 1)) == 0, "TMAX: 1, 2, 4, 8 or 16");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -113,6 +166,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     mbar_init(done, 1);
     fence_barrier_init();
   }
+  __syncwarp();  // warp 0 converged: the CTA barrier counts each warp once
   if (warp == 1) {
     tmem_alloc(tmem_slot, TMEM_COLS);
     tmem_relinquish();
@@ -121,18 +175,19 @@ __global__ void __launch_bounds__(THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  pdl_launch_dependents();  // the next call's kernels may launch and start prefetching
 
   auto stage_a = [&](int s) { return smem + s * STAGE_BYTES; };
   auto stage_b = [&](int s) { return smem + s * STAGE_BYTES + A_BYTES; };
 
   if (warp == 0) {
-    // ------------------------------------------------------------ producer
+    // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       const uint64_t pol = policy_evict_first();
       const int n_units = u1 - u0;
       const int pre = n_units < STAGES ? n_units : STAGES;
-      // The weights do not depend on the preceding kernel: start streaming
-      // them before waiting for it.
+      // The weights do not depend on earlier kernels: stream them before
+      // waiting for the activation codes.
       for (int i = 0; i < pre; ++i) {
         const int u = u0 + i;
         mbar_arrive_expect_tx(&full[i], STAGE_BYTES);
@@ -144,11 +199,9 @@ __global__ void __launch_bounds__(THREADS, 1)
         tma_load_2d(stage_b(i), &tmap_x, &full[i], (u % p.KB) * BK, 0);
       }
       int issued = pre;
-      bool ok = true;
-      for (int i = pre; i < n_units && ok; ++i) {
+      for (int i = pre; i < n_units; ++i) {
         const int s = i % STAGES;
-        ok = mbar_wait(&empty[s], ((i / STAGES) & 1) ^ 1, p.wait_ns, kErrTimeoutProducer);
-        if (!ok) break;
+        if (!mbar_wait(&empty[s], ((i / STAGES) & 1) ^ 1, p.wait_ns, kErrTimeoutProducer)) break;
         const int u = u0 + i;
         mbar_arrive_expect_tx(&full[s], STAGE_BYTES);
         tma_load_2d_hint(stage_a(s), &tmap_w, &full[s], (u % p.KB) * BK, (u / p.KB) * BM, pol);
@@ -203,6 +256,21 @@ __global__ void __launch_bounds__(THREADS, 1)
     const int etid = threadIdx.x - 64;       // 0..127
     const int nO = *p.n_out;
     const int T = p.T;
+    // The outlier product of the (at most two) tiles this CTA shares with
+    // other CTAs does not depend on the int8 accumulators: compute it now,
+    // while the weights stream, so the tile's last CTA only has to combine.
+    const int tile_first = u0 / p.KB, tile_last = (u1 - 1) / p.KB;
+    float yo_first[TMAX], yo_last[TMAX];
+    outlier_product<TMAX>(p, nO, tile_first, row, etid, xo_s, idx_s, yo_first);
+    if (tile_last != tile_first) {
+      outlier_product<TMAX>(p, nO, tile_last, row, etid, xo_s, idx_s, yo_last);
+    } else {
+#pragma unroll
+      for (int t = 0; t < TMAX; ++t) yo_last[t] = yo_first[t];
+    }
+    float sxr[TMAX];
+#pragma unroll
+    for (int t = 0; t < TMAX; ++t) sxr[t] = t < T ? p.sx[t] : 0.0f;
     int seg = 0;
     for (int u = u0; u < u1; ++seg) {
       const int tile = u / p.KB;
@@ -215,6 +283,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       // timeout can never leave some of them at a named barrier.
       const bool ok = mbar_wait(&tfull[buf], (seg >> 1) & 1, p.wait_ns, kErrTimeoutEpilogue);
       if (!named_barrier_and(2, 128, ok)) break;
+      __syncwarp();
       tc_fence_after();
       uint32_t r[16];
       tmem_ld16(tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(buf * NT), r);
@@ -222,18 +291,17 @@ __global__ void __launch_bounds__(THREADS, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&tempty[buf]);
-      int32_t acc[16];
+      int32_t acc[TMAX];
 #pragma unroll
-      for (int t = 0; t < 16; ++t) acc[t] = static_cast<int32_t>(r[t]);
+      for (int t = 0; t < TMAX; ++t) acc[t] = static_cast<int32_t>(r[t]);
 
       if (!whole) {
         const int c_first = cta_of_unit(tile * p.KB, p);
         const int c_last = cta_of_unit((tile + 1) * p.KB - 1, p);
-        const int slot = (tile == u0 / p.KB) ? 0 : 1;
-        int4* mine = reinterpret_cast<int4*>(p.partials +
-                                             (static_cast<int64_t>(cta) * 2 + slot) * SLOT_INTS + row * NT);
+        const int slot = (tile == tile_first) ? 0 : 1;
+        int32_t* mine = p.partials + (static_cast<int64_t>(cta) * 2 + slot) * SLOT_INTS + row * NT;
 #pragma unroll
-        for (int v = 0; v < 4; ++v) mine[v] = make_int4(acc[4 * v], acc[4 * v + 1], acc[4 * v + 2], acc[4 * v + 3]);
+        for (int t = 0; t < TMAX; ++t) mine[t] = acc[t];
         __threadfence();
         named_barrier(1, 128);
         if (etid == 0) {
@@ -243,54 +311,38 @@ __global__ void __launch_bounds__(THREADS, 1)
         named_barrier(1, 128);
         const bool last = *last_flag != 0;
         if (!last) continue;
+        if (etid == 0) p.counters[tile] = 0;  // every contributor has arrived: leave it clean
         __threadfence();
         for (int c2 = c_first; c2 <= c_last; ++c2) {
           if (c2 == cta) continue;
           const int slot2 = (tile == unit_begin(c2, p) / p.KB) ? 0 : 1;
-          const int4* other = reinterpret_cast<const int4*>(
-              p.partials + (static_cast<int64_t>(c2) * 2 + slot2) * SLOT_INTS + row * NT);
+          const int32_t* other = p.partials + (static_cast<int64_t>(c2) * 2 + slot2) * SLOT_INTS + row * NT;
+          int32_t o[TMAX];
 #pragma unroll
-          for (int v = 0; v < 4; ++v) {
-            const int4 o = __ldcg(other + v);
-            acc[4 * v] += o.x;
-            acc[4 * v + 1] += o.y;
-            acc[4 * v + 2] += o.z;
-            acc[4 * v + 3] += o.w;
-          }
+          for (int t = 0; t < TMAX; ++t) o[t] = __ldcg(other + t);
+#pragma unroll
+          for (int t = 0; t < TMAX; ++t) acc[t] += o[t];
         }
       }
 
-      // ---- finalize this tile: outlier product, dequantisation, fp16 store
-      const int n = tile * BM + row;
-      float yo[16];
+      // ---- finalize this tile: dequantisation + outlier product, fp16 store
+      float yo[TMAX];
+      if (tile == tile_first) {
 #pragma unroll
-      for (int t = 0; t < 16; ++t) yo[t] = 0.0f;
-      for (int j0 = 0; j0 < nO; j0 += XO_CHUNK) {
-        const int cnt = min(XO_CHUNK, nO - j0);
-        named_barrier(1, 128);
-        for (int e = etid; e < NT * XO_CHUNK; e += 128) {
-          const int t = e / XO_CHUNK, jj = e % XO_CHUNK;
-          float v = 0.0f;
-          if (t < T && jj < cnt) v = half_bits_to_float(p.X[static_cast<int64_t>(t) * p.K + p.idx[j0 + jj]]);
-          xo_s[e] = v;
-        }
-        if (etid < XO_CHUNK) idx_s[etid] = etid < cnt ? p.idx[j0 + etid] : 0;
-        named_barrier(1, 128);
-        if (n < p.N) {
-          const uint16_t* wrow = p.W + static_cast<int64_t>(n) * p.K;
-          for (int jj = 0; jj < cnt; ++jj) {
-            const float w = half_bits_to_float(__ldg(wrow + idx_s[jj]));
+        for (int t = 0; t < TMAX; ++t) yo[t] = yo_first[t];
+      } else if (tile == tile_last) {
 #pragma unroll
-            for (int t = 0; t < 16; ++t) yo[t] = fmaf(xo_s[t * XO_CHUNK + jj], w, yo[t]);
-          }
-        }
+        for (int t = 0; t < TMAX; ++t) yo[t] = yo_last[t];
+      } else {
+        outlier_product<TMAX>(p, nO, tile, row, etid, xo_s, idx_s, yo);  // a whole tile inside the range
       }
+      const int n = tile * BM + row;
       if (n < p.N) {
         const float swn = p.sw[n];
 #pragma unroll
-        for (int t = 0; t < 16; ++t) {
+        for (int t = 0; t < TMAX; ++t) {
           if (t < T) {
-            const float y = static_cast<float>(acc[t]) * p.sx[t] * swn + yo[t];
+            const float y = static_cast<float>(acc[t]) * sxr[t] * swn + yo[t];
             p.Y[static_cast<int64_t>(t) * p.N + n] = __half_as_ushort(__float2half_rn(y));
             if (p.acc_out) p.acc_out[static_cast<int64_t>(t) * p.N + n] = acc[t];
           }
@@ -299,10 +351,13 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
   }
 
+  // Lane 0 of warps 0 and 1 ran a role loop alone: bring each warp back
+  // together first, so the CTA barrier waits for every warp (an aligned
+  // barrier reached twice by one diverged warp would count it twice).
+  __syncwarp();
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
-    __syncwarp();
     tc_fence_after();
     tmem_dealloc(tmem_base, TMEM_COLS);
   }

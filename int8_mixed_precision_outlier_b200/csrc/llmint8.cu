@@ -59,7 +59,15 @@ int device_info(int* num_sms) {
     }
     if (cudaFuncSetAttribute(gemm::gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              gemm::SMEM_BYTES) != cudaSuccess ||
-        cudaFuncSetAttribute(gemv::gemv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        cudaFuncSetAttribute(gemv::gemv_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             gemv::SMEM_BYTES) != cudaSuccess ||
+        cudaFuncSetAttribute(gemv::gemv_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             gemv::SMEM_BYTES) != cudaSuccess ||
+        cudaFuncSetAttribute(gemv::gemv_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             gemv::SMEM_BYTES) != cudaSuccess ||
+        cudaFuncSetAttribute(gemv::gemv_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             gemv::SMEM_BYTES) != cudaSuccess ||
+        cudaFuncSetAttribute(gemv::gemv_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              gemv::SMEM_BYTES) != cudaSuccess) {
       d.status = LLMINT8_ERR_CUDA;
       return;
@@ -89,11 +97,12 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// 2-D row-major tensor [outer][inner] of `elem_bytes` elements, rows
-// `row_bytes` apart, read in boxes of box_outer rows x box_inner elements
-// (box_inner * elem_bytes == 128: one swizzle row).
+// 2-D row-major tensor [outer][inner], rows `row_bytes` apart, read in boxes
+// of box_outer rows x box_inner elements.  With the 128-byte swizzle a box row
+// is exactly 128 bytes; without swizzle it lands in shared memory row-major.
 bool encode_2d(CUtensorMap* map, CUtensorMapDataType dt, const void* base, uint64_t inner,
-               uint64_t outer, uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer) {
+               uint64_t outer, uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer,
+               CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   const cuuint64_t dims[2] = {inner, outer};
@@ -101,8 +110,8 @@ bool encode_2d(CUtensorMap* map, CUtensorMapDataType dt, const void* base, uint6
   const cuuint32_t box[2] = {box_inner, box_outer};
   const cuuint32_t estr[2] = {1, 1};
   return fn(map, dt, 2, const_cast<void*>(base), dims, strides, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+            CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 // ------------------------------------------------------------ workspace layout
@@ -130,13 +139,12 @@ bool make_layout(int64_t T, int64_t N, int64_t K, int path, Layout* L) {
   };
   if (path == LLMINT8_PATH_GEMV) {
     L->num_tiles = static_cast<int>((N + gemv::BM - 1) / gemv::BM);
-    L->flags = take(sizeof(uint32_t) * L->Kw);
+    L->counters = take(sizeof(int32_t) * (L->num_tiles ? L->num_tiles : 1));
+    L->partials = take(sizeof(int32_t) * gemv::MAX_CTAS * 2 * gemv::SLOT_INTS);
     L->idx = take(sizeof(int32_t) * K);
     L->n_out = take(sizeof(int32_t));
-    L->counters = take(sizeof(int32_t) * (L->num_tiles ? L->num_tiles : 1));
     L->sx = take(sizeof(float) * LLMINT8_GEMV_MAX_T);
     L->xq = take(static_cast<size_t>(LLMINT8_GEMV_MAX_T) * K);
-    L->partials = take(sizeof(int32_t) * gemv::MAX_CTAS * 2 * gemv::SLOT_INTS);
   } else {
     const int64_t strips = (K + kDetectCols - 1) / kDetectCols;
     int64_t R = (kDetectTargetCtas + strips - 1) / strips;
@@ -189,22 +197,24 @@ struct Prep {
   int32_t* n_out;
 };
 
-// Activation stages.  GEMV path: one decode prep kernel.  GEMM path: detect,
-// compact, quantize+gather (the W gather only when W != nullptr).
+// Activation stages.  Decode: one latency-oriented kernel (it also zeroes
+// the GEMV's tile counters when `ncounters` > 0).  Prefill: detect, compact,
+// quantize + gathers (the W gather only when W != nullptr).
 int launch_prep(const Layout& L, const uint16_t* X, int T, int K, const uint16_t* W, int N, float tau,
-                uint8_t* ws, const Prep& out, cudaStream_t st) {
+                uint8_t* ws, const Prep& out, cudaStream_t st, int ncounters = 0) {
   uint32_t* flags = reinterpret_cast<uint32_t*>(ws + L.flags);
   cudaError_t e;
   if (L.path == LLMINT8_PATH_GEMV) {
     int32_t* counters = reinterpret_cast<int32_t*>(ws + L.counters);
-    e = launch(decode_prep_kernel, dim3(1), dim3(kDecodePrepThreads), static_cast<size_t>(K / 8), st,
-               false, X, T, K, tau, flags, out.idx, out.n_out, out.xq, out.sx, counters,
-               W ? L.num_tiles : 0);
+    auto k = T <= 1 ? decode_prep_kernel<1> : T <= 2 ? decode_prep_kernel<2> : T <= 4 ? decode_prep_kernel<4>
+           : T <= 8 ? decode_prep_kernel<8> : decode_prep_kernel<16>;
+    e = launch(k, dim3(1), dim3(kDecodeThreads), 0, st, true, X, T, K, tau, out.xq, out.sx, out.idx,
+               out.n_out, counters, ncounters);
     return e == cudaSuccess ? LLMINT8_OK : LLMINT8_ERR_CUDA;
   }
   uint32_t* part = reinterpret_cast<uint32_t*>(ws + L.part);
   const int strips = (K + kDetectCols - 1) / kDetectCols;
-  e = launch(detect_partial_kernel, dim3(strips, L.R), dim3(kPrepThreads), 0, st, false, X, T, K, tau,
+  e = launch(detect_partial_kernel, dim3(strips, L.R), dim3(kPrepThreads), 0, st, true, X, T, K, tau,
              L.rows_per_chunk, part, L.Kw);
   if (e != cudaSuccess) return LLMINT8_ERR_CUDA;
   e = launch(compact_kernel, dim3(1), dim3(kCompactThreads), 0, st, true,
@@ -232,17 +242,28 @@ int check_common(const void* X, int64_t T, int64_t K, float threshold, const voi
   return LLMINT8_OK;
 }
 
+struct Inspect {  // optional inspection outputs of llmint8_matmul_debug
+  int32_t* acc = nullptr;
+  int8_t* xq = nullptr;
+  float* sx = nullptr;
+  int32_t* idx = nullptr;
+  int32_t* n = nullptr;
+};
+
 int matmul_impl(const void* Xv, int64_t T, int64_t K, const int8_t* Wq, const float* Wscale,
                 const void* Wv, int64_t N, float threshold, void* Yv, void* workspace,
-                size_t ws_bytes, int path, int32_t* acc_out, void* stream,
-                cudaEvent_t ev_begin = nullptr, cudaEvent_t ev_end = nullptr) {
+                size_t ws_bytes, int path, const Inspect& ins, void* stream,
+                cudaEvent_t ev_begin = nullptr, cudaEvent_t ev_end = nullptr, int repeat = 1) {
+  int32_t* acc_out = ins.acc;
   Layout L;
   int rc = check_common(Xv, T, K, threshold, workspace, ws_bytes, path, &L, N);
   if (rc != LLMINT8_OK) return rc;
   if (T == 0 || N == 0) return LLMINT8_OK;
   if (!Wq || !Wscale || !Wv || !Yv) return LLMINT8_ERR_INVALID_ARG;
-  if (!aligned16(Wq) || !aligned16(Wv) || !aligned16(Yv) ||
-      (reinterpret_cast<uintptr_t>(Wscale) & 3u) || (reinterpret_cast<uintptr_t>(acc_out) & 3u))
+  if (!aligned16(Wq) || !aligned16(Wv) || !aligned16(Yv) || !aligned16(ins.xq) ||
+      (reinterpret_cast<uintptr_t>(Wscale) & 3u) || (reinterpret_cast<uintptr_t>(acc_out) & 3u) ||
+      (reinterpret_cast<uintptr_t>(ins.sx) & 3u) || (reinterpret_cast<uintptr_t>(ins.idx) & 3u) ||
+      (reinterpret_cast<uintptr_t>(ins.n) & 3u))
     return LLMINT8_ERR_ALIGNMENT;
   int num_sms = 0;
   rc = device_info(&num_sms);
@@ -254,9 +275,11 @@ int matmul_impl(const void* Xv, int64_t T, int64_t K, const int8_t* Wq, const fl
   uint16_t* Y = static_cast<uint16_t*>(Yv);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   const int t = static_cast<int>(T), n = static_cast<int>(N), k = static_cast<int>(K);
-  Prep out{reinterpret_cast<int8_t*>(ws + L.xq), reinterpret_cast<float*>(ws + L.sx),
-           reinterpret_cast<int32_t*>(ws + L.idx), reinterpret_cast<int32_t*>(ws + L.n_out)};
   const uint64_t wait_ns = g_wait_ns.load();
+  Prep out{ins.xq ? ins.xq : reinterpret_cast<int8_t*>(ws + L.xq),
+           ins.sx ? ins.sx : reinterpret_cast<float*>(ws + L.sx),
+           ins.idx ? ins.idx : reinterpret_cast<int32_t*>(ws + L.idx),
+           ins.n ? ins.n : reinterpret_cast<int32_t*>(ws + L.n_out)};
 
   if (L.path == LLMINT8_PATH_GEMV) {
     gemv::Params p;
@@ -284,12 +307,16 @@ int matmul_impl(const void* Xv, int64_t T, int64_t K, const int8_t* Wq, const fl
     if (!encode_2d(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT8, Wq, K, N, K, gemv::BK, gemv::BM) ||
         !encode_2d(&tx, CU_TENSOR_MAP_DATA_TYPE_UINT8, out.xq, K, T, K, gemv::BK, gemv::NT))
       return LLMINT8_ERR_CUDA;
-    rc = launch_prep(L, X, t, k, W, n, threshold, ws, out, st);
+    rc = launch_prep(L, X, t, k, W, n, threshold, ws, out, st, p.num_tiles);
     if (rc != LLMINT8_OK) return rc;
     if (ev_begin && cudaEventRecord(ev_begin, st) != cudaSuccess) return LLMINT8_ERR_CUDA;
-    cudaError_t e = launch(gemv::gemv_kernel, dim3(grid), dim3(gemv::THREADS), gemv::SMEM_BYTES, st, true,
-                           tw, tx, p);
-    if (e != cudaSuccess) return LLMINT8_ERR_CUDA;
+    void (*kern)(const CUtensorMap, const CUtensorMap, const gemv::Params) =
+        t <= 1 ? gemv::gemv_kernel<1> : t <= 2 ? gemv::gemv_kernel<2> : t <= 4 ? gemv::gemv_kernel<4>
+        : t <= 8 ? gemv::gemv_kernel<8> : gemv::gemv_kernel<16>;
+    for (int r = 0; r < repeat; ++r) {
+      cudaError_t e = launch(kern, dim3(grid), dim3(gemv::THREADS), gemv::SMEM_BYTES, st, true, tw, tx, p);
+      if (e != cudaSuccess) return LLMINT8_ERR_CUDA;
+    }
     if (ev_end && cudaEventRecord(ev_end, st) != cudaSuccess) return LLMINT8_ERR_CUDA;
     return LLMINT8_OK;
   }
@@ -318,9 +345,11 @@ int matmul_impl(const void* Xv, int64_t T, int64_t K, const int8_t* Wq, const fl
   rc = launch_prep(L, X, t, k, W, n, threshold, ws, out, st);
   if (rc != LLMINT8_OK) return rc;
   if (ev_begin && cudaEventRecord(ev_begin, st) != cudaSuccess) return LLMINT8_ERR_CUDA;
-  cudaError_t e = launch(gemm::gemm_kernel, dim3(p.num_m * num_n), dim3(gemm::THREADS), gemm::SMEM_BYTES,
-                         st, true, txq, twq, txo, two, p);
-  if (e != cudaSuccess) return LLMINT8_ERR_CUDA;
+  for (int r = 0; r < repeat; ++r) {
+    cudaError_t e = launch(gemm::gemm_kernel, dim3(p.num_m * num_n), dim3(gemm::THREADS), gemm::SMEM_BYTES,
+                           st, true, txq, twq, txo, two, p);
+    if (e != cudaSuccess) return LLMINT8_ERR_CUDA;
+  }
   if (ev_end && cudaEventRecord(ev_end, st) != cudaSuccess) return LLMINT8_ERR_CUDA;
   return LLMINT8_OK;
 }
@@ -395,22 +424,32 @@ int llmint8_matmul(const void* X, int64_t T, int64_t K, const int8_t* Wq, const 
                    const void* W, int64_t N, float threshold, void* Y, void* workspace,
                    size_t workspace_bytes, void* stream) {
   return matmul_impl(X, T, K, Wq, Wscale, W, N, threshold, Y, workspace, workspace_bytes,
-                     LLMINT8_PATH_AUTO, nullptr, stream);
+                     LLMINT8_PATH_AUTO, Inspect{}, stream);
 }
 
 int llmint8_matmul_debug(const void* X, int64_t T, int64_t K, const int8_t* Wq, const float* Wscale,
                          const void* W, int64_t N, float threshold, void* Y, void* workspace,
-                         size_t workspace_bytes, int path, int32_t* acc_out, void* stream) {
-  return matmul_impl(X, T, K, Wq, Wscale, W, N, threshold, Y, workspace, workspace_bytes, path,
-                     acc_out, stream);
+                         size_t workspace_bytes, int path, int32_t* acc_out, int8_t* xq_out,
+                         float* xscale_out, int32_t* outlier_idx_out, int32_t* n_outliers_out,
+                         void* stream) {
+  Inspect ins;
+  ins.acc = acc_out;
+  ins.xq = xq_out;
+  ins.sx = xscale_out;
+  ins.idx = outlier_idx_out;
+  ins.n = n_outliers_out;
+  return matmul_impl(X, T, K, Wq, Wscale, W, N, threshold, Y, workspace, workspace_bytes, path, ins,
+                     stream);
 }
 
 int llmint8_matmul_profile(const void* X, int64_t T, int64_t K, const int8_t* Wq, const float* Wscale,
                            const void* W, int64_t N, float threshold, void* Y, void* workspace,
-                           size_t workspace_bytes, int path, void* ev_main_begin, void* ev_main_end,
-                           void* stream) {
-  return matmul_impl(X, T, K, Wq, Wscale, W, N, threshold, Y, workspace, workspace_bytes, path, nullptr,
-                     stream, static_cast<cudaEvent_t>(ev_main_begin), static_cast<cudaEvent_t>(ev_main_end));
+                           size_t workspace_bytes, int path, int repeat, void* ev_main_begin,
+                           void* ev_main_end, void* stream) {
+  if (repeat < 1 || repeat > 1000 || !ev_main_begin || !ev_main_end) return LLMINT8_ERR_INVALID_ARG;
+  return matmul_impl(X, T, K, Wq, Wscale, W, N, threshold, Y, workspace, workspace_bytes, path, Inspect{},
+                     stream, static_cast<cudaEvent_t>(ev_main_begin), static_cast<cudaEvent_t>(ev_main_end),
+                     repeat);
 }
 
 int llmint8_detect_quantize(const void* X, int64_t T, int64_t K, float threshold, int8_t* Xq,

@@ -11,61 +11,12 @@
 // division, then round half to even), clamp to [-127, 127], s == 0 -> 0.
 #pragma once
 #include <cuda_fp16.h>
+#include "quant.cuh"
 #include "sm100.cuh"
 
 namespace llmint8 {
 
 constexpr int kPrepThreads = 256;
-
-// Symmetric absmax code of x under scale s.
-__device__ __forceinline__ int8_t quant_code(float x, float s) {
-  if (s == 0.0f) return 0;
-  const float r = __fdiv_rn(x, s);
-  int q = __float2int_rn(r);
-  q = q > 127 ? 127 : (q < -127 ? -127 : q);
-  return static_cast<int8_t>(q);
-}
-
-// Eight halves packed in a uint4 -> their eight codes packed in a uint2.
-// Lanes whose bit is set in `skip` get code 0.
-__device__ __forceinline__ uint2 quant8(const uint4 v, float s, uint32_t skip) {
-  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-  uint32_t out[2] = {0u, 0u};
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const float x = half_bits_to_float(w[i >> 1] >> ((i & 1) * 16));
-    const int8_t q = ((skip >> i) & 1u) ? int8_t(0) : quant_code(x, s);
-    out[i >> 2] |= (static_cast<uint32_t>(static_cast<uint8_t>(q))) << ((i & 3) * 8);
-  }
-  return make_uint2(out[0], out[1]);
-}
-
-// max |x| over the lanes of eight halves whose bit is clear in `skip`.
-__device__ __forceinline__ float absmax8(const uint4 v, uint32_t skip, float m) {
-  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    if ((skip >> i) & 1u) continue;
-    m = fmaxf(m, fabsf(half_bits_to_float(w[i >> 1] >> ((i & 1) * 16))));
-  }
-  return m;
-}
-
-// Bit i set iff |lane i| >= tau.
-__device__ __forceinline__ uint32_t outlier_mask8(const uint4 v, float tau) {
-  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-  uint32_t m = 0;
-#pragma unroll
-  for (int i = 0; i < 8; ++i)
-    m |= (fabsf(half_bits_to_float(w[i >> 1] >> ((i & 1) * 16))) >= tau ? 1u : 0u) << i;
-  return m;
-}
-
-__device__ __forceinline__ float warp_max(float v) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-  return v;
-}
 
 // Block-wide max; `red` is shared scratch of >= 32 floats.
 __device__ __forceinline__ float block_max(float v, float* red) {
@@ -125,9 +76,10 @@ __global__ void __launch_bounds__(kPrepThreads) quantize_weight_kernel(
   for (int c = threadIdx.x; c < nchunk; c += blockDim.x) m = absmax8(__ldg(row + c), 0u, m);
   const float amax = block_max(m, red);
   const float s = __fdiv_rn(amax, 127.0f);
+  const float inv = scale_reciprocal(s);
   if (threadIdx.x == 0) Wscale[n] = s;
   uint2* out = reinterpret_cast<uint2*>(Wq + n * K);
-  for (int c = threadIdx.x; c < nchunk; c += blockDim.x) out[c] = quant8(__ldg(row + c), s, 0u);
+  for (int c = threadIdx.x; c < nchunk; c += blockDim.x) out[c] = quant8(__ldg(row + c), s, inv, 0u);
 }
 
 // ---------------------------------------------------------------------------
@@ -145,6 +97,7 @@ __global__ void __launch_bounds__(kPrepThreads) detect_partial_kernel(
   if (threadIdx.x < 4 * (kDetectCols / 32)) (&words[0][0])[threadIdx.x] = 0u;
   __syncthreads();
   pdl_launch_dependents();
+  pdl_wait();  // X, and the workspace the previous call may still be reading
   const int col0 = blockIdx.x * kDetectCols + c * 8;
   const int t0 = blockIdx.y * rows_per_chunk;
   const int t1 = min(T, t0 + rows_per_chunk);
@@ -185,8 +138,8 @@ __global__ void __launch_bounds__(kCompactThreads) compact_kernel(
     const uint32_t* __restrict__ part, int R, int Kw, uint32_t* __restrict__ flags,
     int32_t* __restrict__ idx, int32_t* __restrict__ n_out) {
   __shared__ int scratch[33];
-  pdl_wait();
   pdl_launch_dependents();
+  pdl_wait();
   const int wpt = (Kw + kCompactThreads - 1) / kCompactThreads;
   const int w0 = threadIdx.x * wpt;
   int count = 0;
@@ -227,8 +180,8 @@ __global__ void __launch_bounds__(kPrepThreads) quant_gather_kernel(
     const int32_t* __restrict__ n_out, int8_t* __restrict__ Xq, float* __restrict__ sx,
     uint16_t* __restrict__ Xo, uint16_t* __restrict__ Wo, int ldo) {
   __shared__ float red[32];
-  pdl_wait();
   pdl_launch_dependents();
+  pdl_wait();
   const int nO = *n_out;
   const int opad = (nO + 63) & ~63;
   if (static_cast<int>(blockIdx.x) < T) {
@@ -240,86 +193,153 @@ __global__ void __launch_bounds__(kPrepThreads) quant_gather_kernel(
     for (int c = threadIdx.x; c < nchunk; c += blockDim.x) m = absmax8(row[c], fb[c], m);
     const float amax = block_max(m, red);
     const float s = __fdiv_rn(amax, 127.0f);
+    const float inv = scale_reciprocal(s);
     if (threadIdx.x == 0) sx[t] = s;
     uint2* out = reinterpret_cast<uint2*>(Xq + t * K);
-    for (int c = threadIdx.x; c < nchunk; c += blockDim.x) out[c] = quant8(row[c], s, fb[c]);
+    for (int c = threadIdx.x; c < nchunk; c += blockDim.x) out[c] = quant8(row[c], s, inv, fb[c]);
     for (int j = threadIdx.x; j < opad; j += blockDim.x)
       Xo[t * ldo + j] = j < nO ? X[t * K + idx[j]] : uint16_t(0);
   } else {
+    // Wo rows: every (row, column) pair is an independent item, 4 loads in
+    // flight per thread before their stores.
     const int64_t n0 = (int64_t)(blockIdx.x - T) * kWoRowsPerCta;
-    for (int rr = 0; rr < kWoRowsPerCta; ++rr) {
-      const int64_t n = n0 + rr;
-      if (n >= N) break;
-      for (int j = threadIdx.x; j < opad; j += blockDim.x)
-        Wo[n * ldo + j] = j < nO ? __ldg(W + n * K + idx[j]) : uint16_t(0);
+    const int64_t left = static_cast<int64_t>(N) - n0;
+    const int rows = left < kWoRowsPerCta ? static_cast<int>(left) : kWoRowsPerCta;
+    const int total = rows * opad;
+    for (int base = threadIdx.x; base < total; base += 4 * blockDim.x) {
+      uint16_t v[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int e = base + u * blockDim.x;
+        v[u] = 0;
+        if (e < total) {
+          const int rr = e / opad, j = e - rr * opad;
+          if (j < nO) v[u] = __ldg(W + (n0 + rr) * K + idx[j]);
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int e = base + u * blockDim.x;
+        if (e < total) {
+          const int rr = e / opad, j = e - rr * opad;
+          Wo[(n0 + rr) * ldo + j] = v[u];
+        }
+      }
     }
   }
 }
 
 // ---------------------------------------------------------------------------
-// Decode (T <= 16): every activation stage in one CTA of 1024 threads --
-// flags, ascending index list, per-row scales and codes -- and the reset of
-// the GEMV's per-tile arrival counters.  Launched without a programmatic
-// dependency, so the previous call on the stream has fully completed; it lets
-// the GEMV launch at once so that the weight stream starts while this runs.
-// Dynamic shared memory: K/8 bytes of per-chunk outlier masks.
+// Decode (T <= 16): every activation stage in one CTA of 1024 threads, built
+// for latency: a pass issues all its loads before using any.  Item e is
+// (chunk c = e / TMAX, row t = e % TMAX) with TMAX = T rounded up to a power of
+// two, so the TMAX rows of a chunk sit in adjacent lanes: its outlier mask is
+// an OR across them, and each thread keeps one row's running absmax.
+//   pass 1: masks -> shared mask bytes; per-row absmax over regular columns
+//   reduce: sx[t] = max / 127, inv[t] = 1 / sx[t]
+//   pass 2: codes (X re-read from L2) -> Xq
+//   then the ascending outlier list, |O|, and zeroed GEMV tile counters.
+// Waits for its predecessor before touching memory and lets the GEMV launch
+// at once, so the GEMV streams weights while this runs.
 // ---------------------------------------------------------------------------
-constexpr int kDecodePrepThreads = 1024;
+constexpr int kDecodeThreads = 1024;
+constexpr int kDecodeInFlight = 8;  // loads per thread per round
 
-__global__ void __launch_bounds__(kDecodePrepThreads) decode_prep_kernel(
-    const uint16_t* __restrict__ X, int T, int K, float tau, uint32_t* __restrict__ flags,
-    int32_t* __restrict__ idx, int32_t* __restrict__ n_out, int8_t* __restrict__ Xq,
-    float* __restrict__ sx, int32_t* __restrict__ counters, int ncounters) {
-  extern __shared__ uint8_t fmask[];  // [K/8]
+template <int TMAX>
+__global__ void __launch_bounds__(kDecodeThreads) decode_prep_kernel(
+    const uint16_t* __restrict__ X, int T, int K, float tau, int8_t* __restrict__ Xq,
+    float* __restrict__ sx, int32_t* __restrict__ idx, int32_t* __restrict__ n_out,
+    int32_t* __restrict__ counters, int ncounters) {
+  __shared__ uint8_t fm[65536 / 8];
+  __shared__ float red[kDecodeThreads / 32][TMAX];
+  __shared__ float s_sx[TMAX], s_inv[TMAX];
   __shared__ int scratch[33];
   pdl_launch_dependents();
+  pdl_wait();
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int nchunk = K >> 3;
-  for (int i = threadIdx.x; i < ncounters; i += blockDim.x) counters[i] = 0;
-  // a1: flags of every 8-column chunk over the T rows
-  for (int c = threadIdx.x; c < nchunk; c += blockDim.x) {
-    uint32_t m = 0;
-    for (int t = 0; t < T; ++t)
-      m |= outlier_mask8(__ldg(reinterpret_cast<const uint4*>(X + (int64_t)t * K) + c), tau);
-    fmask[c] = static_cast<uint8_t>(m);
+  const int items = nchunk * TMAX;
+  const int t = tid % TMAX;
+  const uint16_t* xrow = X + static_cast<int64_t>(t) * K;
+  for (int i = tid; i < ncounters; i += kDecodeThreads) counters[i] = 0;
+
+  // pass 1
+  // rounds are uniform across the block: the shuffles below need whole warps
+  const int rounds = (items + kDecodeThreads * kDecodeInFlight - 1) / (kDecodeThreads * kDecodeInFlight);
+  float m = 0.0f;
+  for (int r = 0; r < rounds; ++r) {
+    const int base = r * kDecodeThreads * kDecodeInFlight + tid;
+    uint4 v[kDecodeInFlight];
+#pragma unroll
+    for (int u = 0; u < kDecodeInFlight; ++u) {
+      const int e = base + u * kDecodeThreads;
+      v[u] = (e < items && t < T) ? __ldg(reinterpret_cast<const uint4*>(xrow) + e / TMAX)
+                                  : make_uint4(0u, 0u, 0u, 0u);
+    }
+#pragma unroll
+    for (int u = 0; u < kDecodeInFlight; ++u) {
+      const int e = base + u * kDecodeThreads;
+      uint32_t mask = outlier_mask8(v[u], tau) & (t < T ? 0xFFu : 0u);
+#pragma unroll
+      for (int o = 1; o < TMAX; o <<= 1) mask |= __shfl_xor_sync(0xffffffffu, mask, o);
+      if (e < items && t == 0) fm[e / TMAX] = static_cast<uint8_t>(mask);
+      m = absmax8(v[u], mask, m);
+    }
+  }
+#pragma unroll
+  for (int o = 16; o >= TMAX; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  if (lane < TMAX) red[warp][lane] = m;
+  __syncthreads();
+  if (tid < TMAX) {
+    float mm = 0.0f;
+    for (int w = 0; w < kDecodeThreads / 32; ++w) mm = fmaxf(mm, red[w][tid]);
+    const float s = __fdiv_rn(mm, 127.0f);
+    s_sx[tid] = s;
+    s_inv[tid] = scale_reciprocal(s);
+    if (tid < T) sx[tid] = s;
   }
   __syncthreads();
-  const int Kw = (K + 31) >> 5;
-  for (int w = threadIdx.x; w < Kw; w += blockDim.x) {
-    uint32_t f = 0;
-    for (int b = 0; b < 4; ++b)
-      if (4 * w + b < nchunk) f |= static_cast<uint32_t>(fmask[4 * w + b]) << (8 * b);
-    flags[w] = f;
+
+  // pass 2
+  const float st = s_sx[t], it = s_inv[t];
+  for (int r = 0; r < rounds; ++r) {
+    const int base = r * kDecodeThreads * kDecodeInFlight + tid;
+    uint4 v[kDecodeInFlight];
+#pragma unroll
+    for (int u = 0; u < kDecodeInFlight; ++u) {
+      const int e = base + u * kDecodeThreads;
+      v[u] = (e < items && t < T) ? __ldg(reinterpret_cast<const uint4*>(xrow) + e / TMAX)
+                                  : make_uint4(0u, 0u, 0u, 0u);
+    }
+#pragma unroll
+    for (int u = 0; u < kDecodeInFlight; ++u) {
+      const int e = base + u * kDecodeThreads;
+      if (e < items && t < T) {
+        const int c = e / TMAX;
+        reinterpret_cast<uint2*>(Xq + static_cast<int64_t>(t) * K)[c] = quant8(v[u], st, it, fm[c]);
+      }
+    }
   }
-  // a4: ascending index list
-  const int cpt = (nchunk + blockDim.x - 1) / blockDim.x;
-  const int c0 = threadIdx.x * cpt;
+
+  // ascending outlier list: thread i owns chunks [i*cpt, (i+1)*cpt)
+  const int cpt = (nchunk + kDecodeThreads - 1) / kDecodeThreads;
+  const int c0 = tid * cpt;
   int count = 0;
   for (int i = 0; i < cpt; ++i)
-    if (c0 + i < nchunk) count += __popc(static_cast<uint32_t>(fmask[c0 + i]));
+    if (c0 + i < nchunk) count += __popc(static_cast<uint32_t>(fm[c0 + i]));
   int total;
   int pos = block_exclusive_scan(count, scratch, &total);
   for (int i = 0; i < cpt; ++i) {
     const int c = c0 + i;
     if (c >= nchunk) break;
-    uint32_t f = fmask[c];
+    uint32_t f = fm[c];
     while (f) {
       const int b = __ffs(f) - 1;
       idx[pos++] = c * 8 + b;
       f &= f - 1;
     }
   }
-  if (threadIdx.x == 0) *n_out = total;
-  // a2 + a3: one warp per row
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  for (int t = warp; t < T; t += blockDim.x >> 5) {
-    const uint4* row = reinterpret_cast<const uint4*>(X + (int64_t)t * K);
-    float m = 0.0f;
-    for (int c = lane; c < nchunk; c += 32) m = absmax8(__ldg(row + c), fmask[c], m);
-    const float s = __fdiv_rn(warp_max(m), 127.0f);
-    if (lane == 0) sx[t] = s;
-    uint2* out = reinterpret_cast<uint2*>(Xq + (int64_t)t * K);
-    for (int c = lane; c < nchunk; c += 32) out[c] = quant8(__ldg(row + c), s, fmask[c]);
-  }
+  if (tid == 0) *n_out = total;
 }
 
 }  // namespace llmint8

@@ -44,8 +44,8 @@ def _declare(lib):
         "llmint8_workspace_bytes": (SZ, [I64, I64, I64]),
         "llmint8_workspace_bytes_path": (SZ, [I64, I64, I64, I]),
         "llmint8_matmul": (I, [P, I64, I64, P, P, P, I64, F, P, P, SZ, P]),
-        "llmint8_matmul_debug": (I, [P, I64, I64, P, P, P, I64, F, P, P, SZ, I, P, P]),
-        "llmint8_matmul_profile": (I, [P, I64, I64, P, P, P, I64, F, P, P, SZ, I, P, P, P]),
+        "llmint8_matmul_debug": (I, [P, I64, I64, P, P, P, I64, F, P, P, SZ, I, P, P, P, P, P, P]),
+        "llmint8_matmul_profile": (I, [P, I64, I64, P, P, P, I64, F, P, P, SZ, I, I, P, P, P]),
         "llmint8_detect_quantize": (I, [P, I64, I64, F, P, P, P, P, P, SZ, I, P]),
         "llmint8_sync_status": (I, [P]),
         "llmint8_selftest_timeout": (I, [U64, P]),
@@ -155,7 +155,9 @@ def llmint8_matmul(X: torch.Tensor, Wq: torch.Tensor, Wscale: torch.Tensor, W: t
 
 def llmint8_matmul_debug(X, Wq, Wscale, W, threshold=6.0, workspace=None, Y=None,
                          path: int = PATH_AUTO, acc_out: torch.Tensor | None = None,
-                         stream=None, _entry: str = "llmint8_matmul_debug"):
+                         stream=None, _entry: str = "llmint8_matmul_debug",
+                         xq_out: torch.Tensor | None = None, sx_out: torch.Tensor | None = None,
+                         idx_out: torch.Tensor | None = None, n_out: torch.Tensor | None = None):
     _need(X, torch.float16, 2, "X")
     _need(Wq, torch.int8, 2, "Wq")
     _need(Wscale, torch.float32, 1, "Wscale")
@@ -171,6 +173,10 @@ def llmint8_matmul_debug(X, Wq, Wscale, W, threshold=6.0, workspace=None, Y=None
         workspace = alloc_workspace(T, N, K, X.device, path)
     if acc_out is not None:
         _need(acc_out, torch.int32, 2, "acc_out")
+    for t, dt, nd, name in ((xq_out, torch.int8, 2, "xq_out"), (sx_out, torch.float32, 1, "sx_out"),
+                            (idx_out, torch.int32, 1, "idx_out"), (n_out, torch.int32, 1, "n_out")):
+        if t is not None:
+            _need(t, dt, nd, name)
     lib = load_library()
     st = _stream(stream)
     if _entry == "llmint8_matmul":
@@ -179,27 +185,49 @@ def llmint8_matmul_debug(X, Wq, Wscale, W, threshold=6.0, workspace=None, Y=None
     else:
         rc = lib.llmint8_matmul_debug(_ptr(X), T, K, _ptr(Wq), _ptr(Wscale), _ptr(W), N,
                                       float(threshold), _ptr(Y), _ptr(workspace),
-                                      workspace.numel(), int(path), _ptr(acc_out), st)
+                                      workspace.numel(), int(path), _ptr(acc_out), _ptr(xq_out),
+                                      _ptr(sx_out), _ptr(idx_out), _ptr(n_out), st)
     _check(rc, _entry)
     return Y
 
 
 def llmint8_matmul_profile(X, Wq, Wscale, W, threshold, workspace, Y, ev_begin, ev_end,
-                           path: int = PATH_AUTO, stream=None):
-    """llmint8_matmul with torch.cuda.Events recorded around the main kernel."""
+                           repeat: int = 1, path: int = PATH_AUTO, stream=None):
+    """Activation stages once, then torch.cuda.Events around `repeat` launches
+    of the main kernel."""
     T, K = X.shape
     N = Wq.shape[0]
+    for ev in (ev_begin, ev_end):
+        if ev.cuda_event == 0:  # torch creates the CUDA event on its first record
+            ev.record()
     rc = load_library().llmint8_matmul_profile(
         _ptr(X), T, K, _ptr(Wq), _ptr(Wscale), _ptr(W), N, float(threshold), _ptr(Y),
-        _ptr(workspace), workspace.numel(), int(path), ctypes.c_void_p(ev_begin.cuda_event),
+        _ptr(workspace), workspace.numel(), int(path), int(repeat), ctypes.c_void_p(ev_begin.cuda_event),
         ctypes.c_void_p(ev_end.cuda_event), _stream(stream))
     _check(rc, "llmint8_matmul_profile")
     return Y
 
 
+def llmint8_matmul_intermediates(X, Wq, Wscale, W, threshold=6.0, path: int = PATH_AUTO,
+                                 workspace=None):
+    """One llmint8_matmul_debug call returning (Y, acc, Xq, sx, outlier_idx)."""
+    T, K = X.shape
+    N = Wq.shape[0]
+    dev = X.device
+    acc = torch.empty((T, N), dtype=torch.int32, device=dev)
+    Xq = torch.empty((T, K), dtype=torch.int8, device=dev)
+    sx = torch.empty(T, dtype=torch.float32, device=dev)
+    idx = torch.empty(K, dtype=torch.int32, device=dev)
+    n = torch.zeros(1, dtype=torch.int32, device=dev)
+    Y = llmint8_matmul_debug(X, Wq, Wscale, W, threshold, workspace, None, path, acc,
+                             xq_out=Xq, sx_out=sx, idx_out=idx, n_out=n)
+    return Y, acc, Xq, sx, idx[: int(n.item())]
+
+
 def llmint8_detect_quantize(X: torch.Tensor, threshold: float = 6.0, path: int = PATH_AUTO,
                             workspace: torch.Tensor | None = None, stream=None):
-    """-> (Xq int8 [T,K], xscale fp32 [T], outlier_idx int32 [|O|])."""
+    """Activation kernels of `path` alone -> (Xq int8 [T,K], xscale fp32 [T],
+    outlier_idx int32 [|O|])."""
     _need(X, torch.float16, 2, "X")
     T, K = X.shape
     dev = X.device
@@ -208,7 +236,7 @@ def llmint8_detect_quantize(X: torch.Tensor, threshold: float = 6.0, path: int =
     idx = torch.empty(K, dtype=torch.int32, device=dev)
     n = torch.zeros(1, dtype=torch.int32, device=dev)
     if workspace is None:
-        workspace = alloc_workspace(T, 1, K, dev, path)
+        workspace = alloc_workspace(T, 0, K, dev, path)
     _check(load_library().llmint8_detect_quantize(
         _ptr(X), T, K, float(threshold), _ptr(Xq), _ptr(sx), _ptr(idx), _ptr(n),
         _ptr(workspace), workspace.numel(), int(path), _stream(stream)), "llmint8_detect_quantize")

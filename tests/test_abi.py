@@ -73,8 +73,14 @@ def test_validation_before_any_device_call(lib):
     assert lib.llmint8_matmul(A, 4, 64, A, A, A, 8, 6.0, A, None, big, None) == -1
     assert lib.llmint8_matmul(A, 4, 64, A, A, A, 8, 6.0, None, A, big, None) == -1
     # bad path; decode path with T > 16
-    assert lib.llmint8_matmul_debug(A, 4, 64, A, A, A, 8, 6.0, A, A, big, 7, None, None) == -1
-    assert lib.llmint8_matmul_debug(A, 17, 64, A, A, A, 8, 6.0, A, A, big, 1, None, None) == -1
+    nil = (None, None, None, None, None)
+    assert lib.llmint8_matmul_debug(A, 4, 64, A, A, A, 8, 6.0, A, A, big, 7, *nil, None) == -1
+    assert lib.llmint8_matmul_debug(A, 17, 64, A, A, A, 8, 6.0, A, A, big, 1, *nil, None) == -1
+    # misaligned inspection output
+    assert lib.llmint8_matmul_debug(A, 4, 64, A, A, A, 8, 6.0, A, A, big, 1, None, _fake(0x10001),
+                                    None, None, None, None) == -2
+    # activation stages alone: the decode path takes T <= 16 only
+    assert lib.llmint8_detect_quantize(A, 17, 64, 6.0, A, A, A, A, A, big, 1, None) == -1
     # K so large that an int32 sum could overflow
     assert lib.llmint8_matmul(A, 4, 140000, A, A, A, 8, 6.0, A, A, big, None) == -1
     # weight quantisation

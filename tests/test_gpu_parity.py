@@ -46,12 +46,11 @@ def run_full(L, oracle, X, W, tau, path):
     Y_o, im = oracle.matmul(X, Wq_o, sw_o, W, tau, intermediates=True)
     Xd, Wd = dev(X), dev(W)
     Wq, sw = L.llmint8_quantize_weight(Wd)
-    T, N = X.shape[0], W.shape[0]
-    acc = torch.empty((T, N), dtype=torch.int32, device="cuda")
-    Y = L.llmint8_matmul_debug(Xd, Wq, sw, Wd, tau, path=path, acc_out=acc)
-    Xq, sx, idx = L.llmint8_detect_quantize(Xd, tau, path=path)
+    Y, acc, Xq, sx, idx = L.llmint8_matmul_intermediates(Xd, Wq, sw, Wd, tau, path=path)
+    Y2 = L.llmint8_matmul_debug(Xd, Wq, sw, Wd, tau, path=path)
     torch.cuda.synchronize()
     ok_status(L)
+    assert_equal(host(Y2), host(Y), "with and without inspection outputs")
     assert_equal(host(Wq), Wq_o, "Wq")
     assert_equal(host(sw).view(np.uint32), sw_o.view(np.uint32), "Wscale")
     assert_equal(host(idx), im["idx"], "outlier idx")
@@ -86,13 +85,28 @@ def test_quantize_weight_worked_example_and_zero_row(L, oracle):
 
 # --------------------------------------------------------------- activations
 
+def activation_stages(L, X, tau, path):
+    """(Xq, sx, idx) of the given path, from the activation kernels alone and
+    from inside a matmul call; the two must agree."""
+    a = L.llmint8_detect_quantize(dev(X), tau, path=path)
+    K = X.shape[1]
+    W = torch.zeros((128, K), dtype=torch.float16, device="cuda")
+    Wq, sw = L.llmint8_quantize_weight(W)
+    _, _, Xq, sx, idx = L.llmint8_matmul_intermediates(dev(X), Wq, sw, W, tau, path=path)
+    torch.cuda.synchronize()
+    assert_equal(host(a[0]), host(Xq), "Xq alone vs in matmul")
+    assert_equal(host(a[1]).view(np.uint32), host(sx).view(np.uint32), "sx alone vs in matmul")
+    assert_equal(host(a[2]), host(idx), "idx alone vs in matmul")
+    return Xq, sx, idx
+
+
 @pytest.mark.parametrize("path,T", [(1, 1), (1, 5), (1, 16), (2, 1), (2, 17), (2, 130), (2, 300)])
 @pytest.mark.parametrize("K", [16, 272, 1040, 4096])
-def test_detect_quantize_bitexact(L, oracle, path, T, K):
+def test_activation_stages_bitexact(L, oracle, path, T, K):
     X, _ = synth.make_activations(T, K, seed=T * 7 + K, n_dims=min(3, K), mag=(6.0, 60.0),
                                   spike_rate=2e-3)
     for tau in (6.0, float("inf"), 0.0, 2.5):
-        Xq, sx, idx = L.llmint8_detect_quantize(dev(X), tau, path=path)
+        Xq, sx, idx = activation_stages(L, X, tau, path)
         flag = oracle.detect_outliers(X, tau)
         Xq_o, sx_o = oracle.quantize_activations(X, flag)
         assert_equal(host(idx), oracle.compact(flag), f"idx tau={tau}")
@@ -110,13 +124,46 @@ def test_detect_edge_values(L, oracle, path):
     X[2, 9] = -6.0
     X[2, 10] = 1.5
     X[3, :] = 0.0                          # zero row: scale 0, codes 0
-    Xq, sx, idx = L.llmint8_detect_quantize(dev(X), 6.0, path=path)
+    Xq, sx, idx = activation_stages(L, X, 6.0, path)
     assert host(idx).tolist() == [3, 9]
     flag = oracle.detect_outliers(X, 6.0)
     Xq_o, sx_o = oracle.quantize_activations(X, flag)
     assert_equal(host(Xq), Xq_o, "Xq")
     assert_equal(host(sx).view(np.uint32), sx_o.view(np.uint32), "sx")
     assert host(sx)[3] == 0.0
+
+
+def near_tie_rows(rng, nrows, K):
+    """Rows of fp16 values whose binary32 quotient x/s lies within 2^-12 of a
+    half-integer (or on it), s = max|row| / 127: the band where a
+    division-free code must defer to the IEEE division."""
+    pos = np.arange(1, 0x7bff, dtype=np.uint16).view(np.float16)
+    rows = []
+    for r in range(nrows):
+        amax = np.float16(127 * 2.0 ** -5) if r % 4 == 0 else np.float16(rng.uniform(0.5, 5.9))
+        s = np.float32(np.float32(amax) / np.float32(127.0))
+        xs = pos[pos.astype(np.float32) < np.float32(amax)]
+        v = xs.astype(np.float32) / s
+        f = v - np.floor(v)
+        near = xs[np.abs(f - np.float32(0.5)) <= np.float32(2.0 ** -12)]
+        assert near.size > 0
+        row = rng.choice(near, K) * np.where(rng.random(K) < 0.5, -1, 1).astype(np.float16)
+        row[rng.integers(0, K)] = amax
+        rows.append(row.astype(np.float16))
+    return np.stack(rows)
+
+
+@pytest.mark.parametrize("path", [1, 2])
+def test_near_tie_codes(L, oracle, path):
+    rng = np.random.default_rng(77 + path)
+    X = near_tie_rows(rng, 16 if path == 1 else 96, 1024)
+    Xq, sx, idx = activation_stages(L, X, float("inf"), path)
+    Xq_o, sx_o = oracle.quantize_activations(X, np.zeros(X.shape[1], np.uint8))
+    assert_equal(host(sx).view(np.uint32), sx_o.view(np.uint32), "sx")
+    assert_equal(host(Xq), Xq_o, "Xq near ties")
+    Wq, sw = L.llmint8_quantize_weight(dev(X))
+    Wq_o, sw_o = oracle.quantize_weight(X)
+    assert_equal(host(Wq), Wq_o, "Wq near ties")
 
 
 # --------------------------------------------------------------- the matmul
@@ -140,7 +187,7 @@ def test_matmul_small(L, oracle, path, T, N, K, tau):
 def test_tiny_config(L, oracle, path):
     w = synth.workload("tiny")
     run_full(L, oracle, w["X"], w["W"], 6.0, path)
-    Xq, sx, idx = L.llmint8_detect_quantize(dev(w["X"]), 6.0, path=path)
+    Xq, sx, idx = activation_stages(L, w["X"], 6.0, path)
     assert host(idx).tolist() == [7, 100]
 
 
@@ -156,11 +203,13 @@ def test_decode_7b_full(L, oracle):
     for T in (1, 2, 4, 8, 16):
         X = np.ascontiguousarray(X16[:T])
         Y_o, im = oracle.matmul(X, Wq_o, sw_o, W, 6.0, intermediates=True)
-        acc = torch.empty((T, W.shape[0]), dtype=torch.int32, device="cuda")
-        Y = L.llmint8_matmul_debug(dev(X), Wq, sw, Wd, 6.0, workspace=ws, path=0, acc_out=acc)
+        Y, acc, Xq, sx, idx = L.llmint8_matmul_intermediates(dev(X), Wq, sw, Wd, 6.0, workspace=ws)
         Y2 = L.llmint8_matmul(dev(X), Wq, sw, Wd, 6.0, workspace=ws)
         torch.cuda.synchronize()
         assert im["nO"] == 4
+        assert_equal(host(idx), im["idx"], f"idx T={T}")
+        assert_equal(host(Xq), im["Xq"], f"Xq T={T}")
+        assert_equal(host(sx).view(np.uint32), im["sx"].view(np.uint32), f"sx T={T}")
         assert_equal(host(acc), im["acc"], f"acc T={T}")
         assert_y_close(host(Y), Y_o, f"Y T={T}")
         assert_equal(host(Y2), host(Y), "debug and plain entry agree")
@@ -290,3 +339,59 @@ def test_int8_linear_wrapper(L, oracle):
     Wq_o, sw_o = oracle.quantize_weight(W)
     assert_y_close(host(Y), oracle.matmul(X, Wq_o, sw_o, W, 6.0), "Y")
     assert_y_close(host(Y1), oracle.matmul(np.ascontiguousarray(X[:1]), Wq_o, sw_o, W, 6.0), "Y1")
+
+
+@pytest.mark.parametrize("path", [1, 2])
+def test_cuda_graph_replay_matches_direct_calls(L, oracle, path):
+    """The calls chain with programmatic dependent launch; captured into a CUDA
+    graph (as the benchmark and a decode loop run them) and replayed, they give
+    the same bytes as direct calls."""
+    T = 16 if path == 1 else 200
+    X, W = synth.random_case(T, 1024, 640, seed=40 + path, n_dims=3)
+    X2, _ = synth.random_case(T, 1024, 640, seed=50 + path, n_dims=5)
+    Wd = dev(W)
+    Wq, sw = L.llmint8_quantize_weight(Wd)
+    ws = L.alloc_workspace(T, 640, 1024, "cuda", path)
+    Xd, X2d = dev(X), dev(X2)
+    Y1 = torch.empty((T, 640), dtype=torch.float16, device="cuda")
+    Y2 = torch.empty_like(Y1)
+    L.llmint8_matmul_debug(Xd, Wq, sw, Wd, 6.0, workspace=ws, Y=Y1, path=path)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        L.llmint8_matmul_debug(Xd, Wq, sw, Wd, 6.0, workspace=ws, Y=Y1, path=path)
+        L.llmint8_matmul_debug(X2d, Wq, sw, Wd, 6.0, workspace=ws, Y=Y2, path=path)
+    Y1.zero_()
+    Y2.zero_()
+    for _ in range(3):
+        g.replay()
+    torch.cuda.synchronize()
+    ok_status(L)
+    Wq_o, sw_o = oracle.quantize_weight(W)
+    assert_y_close(host(Y1), oracle.matmul(X, Wq_o, sw_o, W, 6.0), "graph Y1")
+    assert_y_close(host(Y2), oracle.matmul(X2, Wq_o, sw_o, W, 6.0), "graph Y2")
+    Yd = L.llmint8_matmul_debug(X2d, Wq, sw, Wd, 6.0, workspace=ws, path=path)
+    torch.cuda.synchronize()
+    assert_equal(host(Yd), host(Y2), "graph replay and direct call agree")
+
+
+@pytest.mark.parametrize("path", [1, 2])
+def test_profile_repeats_recompute_same_y(L, oracle, path):
+    """The profiling entry relaunches the main kernel on one workspace; every
+    launch must recompute the same Y (the GEMV's tile counters reset themselves)."""
+    T = 7 if path == 1 else 150
+    X, W = synth.random_case(T, 2048, 700, seed=60 + path, n_dims=4)
+    Wd = dev(W)
+    Wq, sw = L.llmint8_quantize_weight(Wd)
+    ws = L.alloc_workspace(T, 700, 2048, "cuda", path)
+    Y0 = L.llmint8_matmul_debug(dev(X), Wq, sw, Wd, 6.0, workspace=ws, path=path)
+    Y1 = torch.zeros_like(Y0)
+    b = torch.cuda.Event(enable_timing=True)
+    e = torch.cuda.Event(enable_timing=True)
+    L.llmint8_matmul_profile(dev(X), Wq, sw, Wd, 6.0, ws, Y1, b, e, repeat=5, path=path)
+    torch.cuda.synchronize()
+    ok_status(L)
+    assert b.elapsed_time(e) > 0
+    assert_equal(host(Y1), host(Y0), "profile repeats")
+    Wq_o, sw_o = oracle.quantize_weight(W)
+    assert_y_close(host(Y1), oracle.matmul(X, Wq_o, sw_o, W, 6.0), "Y")
