@@ -158,6 +158,27 @@ LLMINT8_API int llmint8_detect_quantize(const void* X, int64_t T, int64_t K, flo
                             void* workspace, size_t workspace_bytes, int path, void* stream);
 
 /*
+ * llmint8_matmul for decode shapes (T <= 16) without a caller workspace and
+ * without allocating anything.  The paper has no counterpart: this entry
+ * serves callers that cannot call cudaMalloc, such as a host program that owns
+ * all device memory through its own pool (a library may not take memory behind
+ * its back) or a latency-critical loop where an allocation could stall the
+ * device or fail mid-run.  Scratch comes from one fixed array in device memory
+ * per GPU that loads the library (5 MiB, kept until the process exits).
+ *   Limits: 1 <= T <= 16, 16 <= K <= 16384, K % 16 == 0, 1 <= N <= 65536;
+ *   larger sizes return LLMINT8_ERR_INVALID_ARG and launch nothing.
+ *   The first call on a device looks up that device's array address (a
+ *   runtime symbol query); later calls only launch kernels.
+ *   Every call on a device shares the array and leaves its contents behind, so
+ *   calls must not overlap on the GPU: order them on one stream, or two
+ *   overlapping calls race on the scratch and both results are undefined.
+ * Arguments, layouts and results are those of llmint8_matmul.
+ */
+LLMINT8_API int llmint8_matmul_decode_noalloc(const void* X, int64_t T, int64_t K, const int8_t* Wq,
+                                              const float* Wscale, const void* W, int64_t N,
+                                              float threshold, void* Y, void* stream);
+
+/*
  * Waits for `stream`, then reads and clears this device's error word.
  * Returns LLMINT8_ERR_TIMEOUT if a kernel gave up a bounded wait since the
  * last call, LLMINT8_ERR_CUDA if the stream reported an error, else OK.

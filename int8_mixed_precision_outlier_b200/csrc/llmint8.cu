@@ -354,6 +354,36 @@ int matmul_impl(const void* Xv, int64_t T, int64_t K, const int8_t* Wq, const fl
   return LLMINT8_OK;
 }
 
+// ------------------------------------------------------------ allocation-free decode
+// Scratch for llmint8_matmul_decode_noalloc: one array per device that loads
+// the library, held until the process exits.  Sized for the decode path's
+// workspace at T <= 16, K <= kNoAllocMaxK, N <= kNoAllocMaxN (about 4.4 MB
+// used of 5 MiB; the stream-K partial slots are most of it).
+constexpr int64_t kNoAllocMaxK = 16384;
+constexpr int64_t kNoAllocMaxN = 65536;
+constexpr size_t kNoAllocScratchBytes = 5u << 20;
+static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
+
+struct NoAllocScratch {
+  std::once_flag once;
+  void* ptr = nullptr;
+  cudaError_t err = cudaSuccess;
+};
+NoAllocScratch g_noalloc[kMaxDevices];
+
+// Device address of this device's scratch array.  In host code the array's
+// name stands for a host-side shadow, not device memory, so the address is
+// queried once per device, with that device current.
+int noalloc_scratch(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return LLMINT8_ERR_CUDA;
+  NoAllocScratch& d = g_noalloc[dev];
+  std::call_once(d.once, [&]() { d.err = cudaGetSymbolAddress(&d.ptr, g_noalloc_scratch); });
+  if (d.err != cudaSuccess || d.ptr == nullptr) return LLMINT8_ERR_CUDA;
+  *out = d.ptr;
+  return LLMINT8_OK;
+}
+
 __global__ void selftest_timeout_kernel(uint64_t wait_ns) {
   __shared__ uint64_t bar;
   if (threadIdx.x == 0) {
@@ -469,6 +499,26 @@ int llmint8_detect_quantize(const void* X, int64_t T, int64_t K, float threshold
   Prep out{Xq, xscale, outlier_idx, n_outliers};
   return launch_prep(L, static_cast<const uint16_t*>(X), static_cast<int>(T), static_cast<int>(K), nullptr,
                      0, threshold, static_cast<uint8_t*>(workspace), out, static_cast<cudaStream_t>(stream));
+}
+
+int llmint8_matmul_decode_noalloc(const void* X, int64_t T, int64_t K, const int8_t* Wq,
+                                  const float* Wscale, const void* W, int64_t N, float threshold,
+                                  void* Y, void* stream) {
+  if (T < 0 || T > LLMINT8_GEMV_MAX_T || K > kNoAllocMaxK || N < 0 || N > kNoAllocMaxN)
+    return LLMINT8_ERR_INVALID_ARG;
+  Layout L;
+  if (!make_layout(T, N, K, LLMINT8_PATH_GEMV, &L)) return LLMINT8_ERR_INVALID_ARG;
+  if (L.total > kNoAllocScratchBytes) return LLMINT8_ERR_WORKSPACE;
+  if (T == 0 || N == 0) return LLMINT8_OK;
+  int rc = device_info(nullptr);
+  if (rc != LLMINT8_OK) return rc;
+  void* scratch = nullptr;
+  rc = noalloc_scratch(&scratch);
+  if (rc != LLMINT8_OK) return rc;
+  // The decode prep kernel zeroes the per-tile counters at the start of every
+  // call; every other scratch word is written before it is read.
+  return matmul_impl(X, T, K, Wq, Wscale, W, N, threshold, Y, scratch, kNoAllocScratchBytes,
+                     LLMINT8_PATH_GEMV, Inspect{}, stream);
 }
 
 int llmint8_sync_status(void* stream) {

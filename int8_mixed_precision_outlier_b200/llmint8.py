@@ -47,6 +47,7 @@ def _declare(lib):
         "llmint8_matmul_debug": (I, [P, I64, I64, P, P, P, I64, F, P, P, SZ, I, P, P, P, P, P, P]),
         "llmint8_matmul_profile": (I, [P, I64, I64, P, P, P, I64, F, P, P, SZ, I, I, P, P, P]),
         "llmint8_detect_quantize": (I, [P, I64, I64, F, P, P, P, P, P, SZ, I, P]),
+        "llmint8_matmul_decode_noalloc": (I, [P, I64, I64, P, P, P, I64, F, P, P]),
         "llmint8_sync_status": (I, [P]),
         "llmint8_selftest_timeout": (I, [U64, P]),
         "llmint8_set_wait_limit_ns": (I, [U64]),
@@ -151,6 +152,27 @@ def llmint8_matmul(X: torch.Tensor, Wq: torch.Tensor, Wscale: torch.Tensor, W: t
     """Y = X W^T by the LLM.int8() decomposition (fp16 [T,N])."""
     return llmint8_matmul_debug(X, Wq, Wscale, W, threshold, workspace, Y, PATH_AUTO, None,
                                 stream, _entry="llmint8_matmul")
+
+
+def llmint8_matmul_decode_noalloc(X: torch.Tensor, Wq: torch.Tensor, Wscale: torch.Tensor,
+                                  W: torch.Tensor, threshold: float = 6.0,
+                                  Y: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Decode-shaped Y = X W^T (T <= 16) with no workspace: the library's scratch
+    is a fixed per-GPU array, for callers that must not allocate device memory.
+    Calls must not overlap on the GPU (they share that array)."""
+    _need(X, torch.float16, 2, "X")
+    _need(Wq, torch.int8, 2, "Wq")
+    _need(Wscale, torch.float32, 1, "Wscale")
+    _need(W, torch.float16, 2, "W")
+    T, K = X.shape
+    N = Wq.shape[0]
+    if Y is None:
+        Y = torch.empty((T, N), dtype=torch.float16, device=X.device)
+    _need(Y, torch.float16, 2, "Y")
+    _check(load_library().llmint8_matmul_decode_noalloc(
+        _ptr(X), T, K, _ptr(Wq), _ptr(Wscale), _ptr(W), N, float(threshold), _ptr(Y),
+        _stream(stream)), "llmint8_matmul_decode_noalloc")
+    return Y
 
 
 def llmint8_matmul_debug(X, Wq, Wscale, W, threshold=6.0, workspace=None, Y=None,
