@@ -37,7 +37,7 @@ namespace gemv {
 constexpr int BM = 128;                    // weight rows per tile = MMA M
 constexpr int BK = 128;                    // K bytes per k-block (one 128 B swizzle row)
 constexpr int NT = 16;                     // tokens per MMA (MMA N)
-constexpr int STAGES = 8;
+constexpr int STAGES = 11;
 constexpr int A_BYTES = BM * BK;           // 16 KiB of Wq
 constexpr int B_BYTES = NT * BK;           // 2 KiB of activation codes
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
@@ -80,17 +80,25 @@ __device__ __forceinline__ int cta_of_unit(int u, const Params& p) {
   return c;
 }
 
-// yo[t] = sum_{j<|O|} X[t, O_j] * W[n, O_j] (fp32, ascending j) for the tile row
-// n = tile * BM + row, t < TMAX (zero past T).  All 128 epilogue threads call
-// this together: they stage X's outlier values of 64 columns at a time in
-// shared memory, then each thread gathers its row's weights 8 at a time so
-// that the loads are in flight together.
+// Outlier products of one tile row in each of two tiles (the two may be the
+// same): for n = tile * BM + row,
+//   yo[t] = sum_{j<|O|} X[t, O_j] * W[n, O_j]   (fp32, ascending j), t < TMAX.
+// All 128 epilogue threads call this together.  Per 64 outlier columns: the
+// indices go to shared memory, then the X values and both rows' W values are
+// gathered with all loads in flight at once (two dependent round trips per
+// chunk, whatever the number of tiles).
 template <int TMAX>
-__device__ __forceinline__ void outlier_product(const Params& p, int nO, int tile, int row, int etid,
-                                                float* xo_s, int32_t* idx_s, float (&yo)[TMAX]) {
+__device__ __forceinline__ void outlier_products(const Params& p, int nO, int tile_a, int tile_b, int row,
+                                                 int etid, float* xo_s, int32_t* idx_s, float (&ya)[TMAX],
+                                                 float (&yb)[TMAX]) {
 #pragma unroll
-  for (int t = 0; t < TMAX; ++t) yo[t] = 0.0f;
-  const int n = tile * BM + row;
+  for (int t = 0; t < TMAX; ++t) {
+    ya[t] = 0.0f;
+    yb[t] = 0.0f;
+  }
+  const int na = tile_a * BM + row, nb = tile_b * BM + row;
+  const uint16_t* wa = p.W + static_cast<int64_t>(na < p.N ? na : 0) * p.K;
+  const uint16_t* wb = p.W + static_cast<int64_t>(nb < p.N ? nb : 0) * p.K;
   for (int j0 = 0; j0 < nO; j0 += XO_CHUNK) {
     const int cnt = min(XO_CHUNK, nO - j0);
     named_barrier(1, 128);  // the previous chunk has been read
@@ -106,21 +114,36 @@ __device__ __forceinline__ void outlier_product(const Params& p, int nO, int til
                  ? half_bits_to_float(p.X[static_cast<int64_t>(t) * p.K + idx_s[jj]])
                  : 0.0f;
     }
+    constexpr int G = 8;  // outlier columns per batch of weight loads
+    uint16_t w_a[G], w_b[G];
+#pragma unroll
+    for (int u = 0; u < G; ++u) {
+      const int k = u < cnt ? idx_s[u] : 0;
+      w_a[u] = u < cnt ? __ldg(wa + k) : uint16_t(0);
+      w_b[u] = u < cnt ? __ldg(wb + k) : uint16_t(0);
+    }
 #pragma unroll
     for (int i = 0; i < PER; ++i)
       if (etid + 128 * i < TMAX * XO_CHUNK) xo_s[etid + 128 * i] = v[i];
     named_barrier(1, 128);
-    if (n < p.N) {
-      const uint16_t* wrow = p.W + static_cast<int64_t>(n) * p.K;
-      for (int jj0 = 0; jj0 < cnt; jj0 += 8) {
-        float w[8];
+    for (int jj0 = 0; jj0 < cnt; jj0 += G) {
+      if (jj0 > 0) {
 #pragma unroll
-        for (int u = 0; u < 8; ++u)
-          w[u] = (jj0 + u < cnt) ? half_bits_to_float(__ldg(wrow + idx_s[jj0 + u])) : 0.0f;
+        for (int u = 0; u < G; ++u) {
+          const int k = jj0 + u < cnt ? idx_s[jj0 + u] : 0;
+          w_a[u] = jj0 + u < cnt ? __ldg(wa + k) : uint16_t(0);
+          w_b[u] = jj0 + u < cnt ? __ldg(wb + k) : uint16_t(0);
+        }
+      }
 #pragma unroll
-        for (int u = 0; u < 8; ++u)
+      for (int u = 0; u < G; ++u) {
+        const float fa = half_bits_to_float(w_a[u]), fb = half_bits_to_float(w_b[u]);
 #pragma unroll
-          for (int t = 0; t < TMAX; ++t) yo[t] = fmaf(xo_s[t * XO_CHUNK + jj0 + u], w[u], yo[t]);
+        for (int t = 0; t < TMAX; ++t) {
+          const float x = xo_s[t * XO_CHUNK + jj0 + u];
+          ya[t] = fmaf(x, fa, ya[t]);
+          yb[t] = fmaf(x, fb, yb[t]);
+        }
       }
     }
   }
@@ -261,13 +284,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     // while the weights stream, so the tile's last CTA only has to combine.
     const int tile_first = u0 / p.KB, tile_last = (u1 - 1) / p.KB;
     float yo_first[TMAX], yo_last[TMAX];
-    outlier_product<TMAX>(p, nO, tile_first, row, etid, xo_s, idx_s, yo_first);
-    if (tile_last != tile_first) {
-      outlier_product<TMAX>(p, nO, tile_last, row, etid, xo_s, idx_s, yo_last);
-    } else {
-#pragma unroll
-      for (int t = 0; t < TMAX; ++t) yo_last[t] = yo_first[t];
-    }
+    outlier_products<TMAX>(p, nO, tile_first, tile_last, row, etid, xo_s, idx_s, yo_first, yo_last);
     float sxr[TMAX];
 #pragma unroll
     for (int t = 0; t < TMAX; ++t) sxr[t] = t < T ? p.sx[t] : 0.0f;
@@ -302,17 +319,22 @@ __global__ void __launch_bounds__(THREADS, 1)
         int32_t* mine = p.partials + (static_cast<int64_t>(cta) * 2 + slot) * SLOT_INTS + row * NT;
 #pragma unroll
         for (int t = 0; t < TMAX; ++t) mine[t] = acc[t];
-        __threadfence();
+        // The barrier orders the 128 threads' stores before the signalling
+        // thread's GPU-scope fence (cumulativity), which releases them all
+        // with its counter update; the last arriver's fence acquires the
+        // others' partials, and the second barrier passes that on.
         named_barrier(1, 128);
         if (etid == 0) {
+          __threadfence();
           const int old = atomicAdd(&p.counters[tile], 1);
-          *last_flag = (old == c_last - c_first) ? 1 : 0;
+          __threadfence();
+          const bool is_last = old == c_last - c_first;
+          if (is_last) p.counters[tile] = 0;  // every contributor has arrived: leave it clean
+          *last_flag = is_last ? 1 : 0;
         }
         named_barrier(1, 128);
         const bool last = *last_flag != 0;
         if (!last) continue;
-        if (etid == 0) p.counters[tile] = 0;  // every contributor has arrived: leave it clean
-        __threadfence();
         for (int c2 = c_first; c2 <= c_last; ++c2) {
           if (c2 == cta) continue;
           const int slot2 = (tile == unit_begin(c2, p) / p.KB) ? 0 : 1;
@@ -334,7 +356,8 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
         for (int t = 0; t < TMAX; ++t) yo[t] = yo_last[t];
       } else {
-        outlier_product<TMAX>(p, nO, tile, row, etid, xo_s, idx_s, yo);  // a whole tile inside the range
+        float unused[TMAX];
+        outlier_products<TMAX>(p, nO, tile, tile, row, etid, xo_s, idx_s, yo, unused);  // a whole tile
       }
       const int n = tile * BM + row;
       if (n < p.N) {

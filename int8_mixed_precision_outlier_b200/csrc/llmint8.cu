@@ -172,21 +172,40 @@ bool make_layout(int64_t T, int64_t N, int64_t K, int path, Layout* L) {
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 // ------------------------------------------------------------ launches
+// Launch with programmatic stream serialization (when `pdl`) and, when
+// `cluster` > 1, thread-block clusters of that many CTAs along x.
 template <typename... Exp, typename... Act>
-cudaError_t launch(void (*kern)(Exp...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, bool pdl,
-                   Act&&... args) {
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
+cudaError_t launch_ex(void (*kern)(Exp...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, bool pdl,
+                      int cluster, Act&&... args) {
+  cudaLaunchAttribute attr[2];
+  int n = 0;
+  if (pdl) {
+    attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[n].val.programmaticStreamSerializationAllowed = 1;
+    ++n;
+  }
+  if (cluster > 1) {
+    attr[n].id = cudaLaunchAttributeClusterDimension;
+    attr[n].val.clusterDim.x = static_cast<unsigned>(cluster);
+    attr[n].val.clusterDim.y = 1;
+    attr[n].val.clusterDim.z = 1;
+    ++n;
+  }
   cudaLaunchConfig_t cfg;
   std::memset(&cfg, 0, sizeof(cfg));
   cfg.gridDim = grid;
   cfg.blockDim = block;
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
-  cfg.attrs = pdl ? attr : nullptr;
-  cfg.numAttrs = pdl ? 1 : 0;
+  cfg.attrs = n ? attr : nullptr;
+  cfg.numAttrs = n;
   return cudaLaunchKernelEx(&cfg, kern, std::forward<Act>(args)...);
+}
+
+template <typename... Exp, typename... Act>
+cudaError_t launch(void (*kern)(Exp...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, bool pdl,
+                   Act&&... args) {
+  return launch_ex(kern, grid, block, smem, st, pdl, 1, std::forward<Act>(args)...);
 }
 
 struct Prep {
@@ -208,8 +227,8 @@ int launch_prep(const Layout& L, const uint16_t* X, int T, int K, const uint16_t
     int32_t* counters = reinterpret_cast<int32_t*>(ws + L.counters);
     auto k = T <= 1 ? decode_prep_kernel<1> : T <= 2 ? decode_prep_kernel<2> : T <= 4 ? decode_prep_kernel<4>
            : T <= 8 ? decode_prep_kernel<8> : decode_prep_kernel<16>;
-    e = launch(k, dim3(1), dim3(kDecodeThreads), 0, st, true, X, T, K, tau, out.xq, out.sx, out.idx,
-               out.n_out, counters, ncounters);
+    e = launch_ex(k, dim3(kDecodeCtas), dim3(kDecodeThreads), 0, st, true, kDecodeCtas, X, T, K, tau, out.xq,
+                  out.sx, out.idx, out.n_out, counters, ncounters);
     return e == cudaSuccess ? LLMINT8_OK : LLMINT8_ERR_CUDA;
   }
   uint32_t* part = reinterpret_cast<uint32_t*>(ws + L.part);

@@ -230,51 +230,64 @@ __global__ void __launch_bounds__(kPrepThreads) quant_gather_kernel(
 }
 
 // ---------------------------------------------------------------------------
-// Decode (T <= 16): every activation stage in one CTA of 1024 threads, built
-// for latency: a pass issues all its loads before using any.  Item e is
-// (chunk c = e / TMAX, row t = e % TMAX) with TMAX = T rounded up to a power of
-// two, so the TMAX rows of a chunk sit in adjacent lanes: its outlier mask is
-// an OR across them, and each thread keeps one row's running absmax.
+// Decode (T <= 16): every activation stage in one cluster of 8 CTAs.  CTA r of
+// the cluster owns a contiguous slice of 8-column chunks for all T rows.  Item
+// e of a CTA is (chunk c = e / TMAX, row t = e % TMAX), TMAX = T rounded up to a
+// power of two, so a chunk's rows sit in adjacent lanes: its outlier mask is an
+// OR across them, and each thread keeps one row's running absmax.
 //   pass 1: masks -> shared mask bytes; per-row absmax over regular columns
-//   reduce: sx[t] = max / 127, inv[t] = 1 / sx[t]
-//   pass 2: codes (X re-read from L2) -> Xq
-//   then the ascending outlier list, |O|, and zeroed GEMV tile counters.
-// Waits for its predecessor before touching memory and lets the GEMV launch
-// at once, so the GEMV streams weights while this runs.
+//   exchange: each CTA writes its per-row maxima and its outlier count into
+//     rank 0's shared memory (distributed shared memory); after a cluster
+//     barrier every CTA forms sx[t] = max / 127 and its offset in the list
+//   pass 2: codes (X re-read from L2) -> Xq; this CTA's outlier indices
+// 256 threads and at most 64 registers per CTA let a CTA share an SM with a
+// GEMV CTA, so the cluster launches while the previous call's GEMV runs.  It
+// waits for its predecessor before touching memory and lets the GEMV launch at
+// once, so the GEMV streams weights while this runs.
 // ---------------------------------------------------------------------------
-constexpr int kDecodeThreads = 1024;
-constexpr int kDecodeInFlight = 8;  // loads per thread per round
+constexpr int kDecodeCtas = 8;
+constexpr int kDecodeThreads = 256;
+constexpr int kDecodeInFlight = 4;   // loads per thread per round
+constexpr int kDecodeMaxSlice = 65536 / 8 / kDecodeCtas;  // chunks per CTA at K = 65536
 
 template <int TMAX>
-__global__ void __launch_bounds__(kDecodeThreads) decode_prep_kernel(
+__global__ void __launch_bounds__(kDecodeThreads, 4) decode_prep_kernel(
     const uint16_t* __restrict__ X, int T, int K, float tau, int8_t* __restrict__ Xq,
     float* __restrict__ sx, int32_t* __restrict__ idx, int32_t* __restrict__ n_out,
     int32_t* __restrict__ counters, int ncounters) {
-  __shared__ uint8_t fm[65536 / 8];
+  __shared__ uint8_t fm[kDecodeMaxSlice];
   __shared__ float red[kDecodeThreads / 32][TMAX];
+  __shared__ float part[kDecodeCtas][TMAX];  // read in rank 0: every CTA's row maxima
+  __shared__ int cnt[kDecodeCtas];           // read in rank 0: every CTA's outlier count
   __shared__ float s_sx[TMAX], s_inv[TMAX];
+  __shared__ int s_off;
   __shared__ int scratch[33];
   pdl_launch_dependents();
+  cluster_sync();  // every CTA of the cluster has started before any remote access
   pdl_wait();
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const uint32_t rank = cluster_ctarank();
   const int nchunk = K >> 3;
-  const int items = nchunk * TMAX;
+  const int cpc = (nchunk + kDecodeCtas - 1) / kDecodeCtas;
+  const int c_begin = static_cast<int>(rank) * cpc;
+  const int myn = max(0, min(nchunk, c_begin + cpc) - c_begin);
+  const int items = myn * TMAX;
   const int t = tid % TMAX;
-  const uint16_t* xrow = X + static_cast<int64_t>(t) * K;
-  for (int i = tid; i < ncounters; i += kDecodeThreads) counters[i] = 0;
+  const uint4* xrow = reinterpret_cast<const uint4*>(X + static_cast<int64_t>(t) * K) + c_begin;
+  for (int i = static_cast<int>(rank) * kDecodeThreads + tid; i < ncounters; i += kDecodeCtas * kDecodeThreads)
+    counters[i] = 0;
 
-  // pass 1
-  // rounds are uniform across the block: the shuffles below need whole warps
+  // pass 1 (rounds are uniform across the CTA: the shuffles need whole warps)
   const int rounds = (items + kDecodeThreads * kDecodeInFlight - 1) / (kDecodeThreads * kDecodeInFlight);
   float m = 0.0f;
+  uint4 keep[kDecodeInFlight];  // the slice's values when one round covers it
   for (int r = 0; r < rounds; ++r) {
     const int base = r * kDecodeThreads * kDecodeInFlight + tid;
     uint4 v[kDecodeInFlight];
 #pragma unroll
     for (int u = 0; u < kDecodeInFlight; ++u) {
       const int e = base + u * kDecodeThreads;
-      v[u] = (e < items && t < T) ? __ldg(reinterpret_cast<const uint4*>(xrow) + e / TMAX)
-                                  : make_uint4(0u, 0u, 0u, 0u);
+      v[u] = (e < items && t < T) ? __ldg(xrow + e / TMAX) : make_uint4(0u, 0u, 0u, 0u);
     }
 #pragma unroll
     for (int u = 0; u < kDecodeInFlight; ++u) {
@@ -284,21 +297,46 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_prep_kernel(
       for (int o = 1; o < TMAX; o <<= 1) mask |= __shfl_xor_sync(0xffffffffu, mask, o);
       if (e < items && t == 0) fm[e / TMAX] = static_cast<uint8_t>(mask);
       m = absmax8(v[u], mask, m);
+      keep[u] = v[u];
     }
   }
 #pragma unroll
   for (int o = 16; o >= TMAX; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
   if (lane < TMAX) red[warp][lane] = m;
   __syncthreads();
+  int count = 0;
+  for (int i = tid; i < myn; i += kDecodeThreads) count += __popc(static_cast<uint32_t>(fm[i]));
+  int my_total;
+  block_exclusive_scan(count, scratch, &my_total);
+  if (tid < TMAX) {
+    float pm = 0.0f;
+#pragma unroll
+    for (int w = 0; w < kDecodeThreads / 32; ++w) pm = fmaxf(pm, red[w][tid]);
+    st_cluster_f32(map_shared_rank(&part[rank][tid], 0), pm);
+  }
+  if (tid == 0) st_cluster_u32(map_shared_rank(&cnt[rank], 0), static_cast<uint32_t>(my_total));
+  cluster_sync();
+
   if (tid < TMAX) {
     float mm = 0.0f;
-    for (int w = 0; w < kDecodeThreads / 32; ++w) mm = fmaxf(mm, red[w][tid]);
+#pragma unroll
+    for (int r = 0; r < kDecodeCtas; ++r) mm = fmaxf(mm, ld_cluster_f32(map_shared_rank(&part[r][tid], 0)));
     const float s = __fdiv_rn(mm, 127.0f);
     s_sx[tid] = s;
     s_inv[tid] = scale_reciprocal(s);
-    if (tid < T) sx[tid] = s;
+    if (rank == 0 && tid < T) sx[tid] = s;
   }
-  __syncthreads();
+  if (tid == 32) {
+    int off = 0, total = 0;
+    for (int r = 0; r < kDecodeCtas; ++r) {
+      const int c = static_cast<int>(ld_cluster_u32(map_shared_rank(&cnt[r], 0)));
+      off += r < static_cast<int>(rank) ? c : 0;
+      total += c;
+    }
+    s_off = off;
+    if (rank == 0) *n_out = total;
+  }
+  cluster_sync();  // rank 0's shared memory stays valid until every CTA has read it
 
   // pass 2
   const float st = s_sx[t], it = s_inv[t];
@@ -308,38 +346,37 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_prep_kernel(
 #pragma unroll
     for (int u = 0; u < kDecodeInFlight; ++u) {
       const int e = base + u * kDecodeThreads;
-      v[u] = (e < items && t < T) ? __ldg(reinterpret_cast<const uint4*>(xrow) + e / TMAX)
-                                  : make_uint4(0u, 0u, 0u, 0u);
+      v[u] = rounds == 1 ? keep[u]
+             : (e < items && t < T) ? __ldg(xrow + e / TMAX) : make_uint4(0u, 0u, 0u, 0u);
     }
 #pragma unroll
     for (int u = 0; u < kDecodeInFlight; ++u) {
       const int e = base + u * kDecodeThreads;
       if (e < items && t < T) {
         const int c = e / TMAX;
-        reinterpret_cast<uint2*>(Xq + static_cast<int64_t>(t) * K)[c] = quant8(v[u], st, it, fm[c]);
+        reinterpret_cast<uint2*>(Xq + static_cast<int64_t>(t) * K)[c_begin + c] = quant8(v[u], st, it, fm[c]);
       }
     }
   }
 
-  // ascending outlier list: thread i owns chunks [i*cpt, (i+1)*cpt)
-  const int cpt = (nchunk + kDecodeThreads - 1) / kDecodeThreads;
+  // this CTA's outlier indices, ascending: thread i owns chunks [i*cpt, (i+1)*cpt)
+  const int cpt = (myn + kDecodeThreads - 1) / kDecodeThreads;
   const int c0 = tid * cpt;
-  int count = 0;
+  count = 0;
   for (int i = 0; i < cpt; ++i)
-    if (c0 + i < nchunk) count += __popc(static_cast<uint32_t>(fm[c0 + i]));
-  int total;
-  int pos = block_exclusive_scan(count, scratch, &total);
+    if (c0 + i < myn) count += __popc(static_cast<uint32_t>(fm[c0 + i]));
+  int unused;
+  int pos = s_off + block_exclusive_scan(count, scratch, &unused);
   for (int i = 0; i < cpt; ++i) {
     const int c = c0 + i;
-    if (c >= nchunk) break;
+    if (c >= myn) break;
     uint32_t f = fm[c];
     while (f) {
       const int b = __ffs(f) - 1;
-      idx[pos++] = c * 8 + b;
+      idx[pos++] = (c_begin + c) * 8 + b;
       f &= f - 1;
     }
   }
-  if (tid == 0) *n_out = total;
 }
 
 }  // namespace llmint8
