@@ -240,10 +240,10 @@ int launch_prep(const Layout& L, const uint16_t* X, int T, int K, const uint16_t
              static_cast<const uint32_t*>(part), L.R, L.Kw, flags, out.idx, out.n_out);
   if (e != cudaSuccess) return LLMINT8_ERR_CUDA;
   const int wblocks = W ? (N + kWoRowsPerCta - 1) / kWoRowsPerCta : 0;
-  e = launch(quant_gather_kernel, dim3(T + wblocks), dim3(kPrepThreads), 0, st, true, X, T, K, W, N,
+  e = launch(quant_gather_kernel, dim3(wblocks + T), dim3(kQuantThreads), 0, st, true, X, T, K, W, N,
              static_cast<const uint32_t*>(flags), static_cast<const int32_t*>(out.idx),
              static_cast<const int32_t*>(out.n_out), out.xq, out.sx,
-             reinterpret_cast<uint16_t*>(ws + L.xo), reinterpret_cast<uint16_t*>(ws + L.wo), L.ldo);
+             reinterpret_cast<uint16_t*>(ws + L.xo), reinterpret_cast<uint16_t*>(ws + L.wo), L.ldo, wblocks);
   return e == cudaSuccess ? LLMINT8_OK : LLMINT8_ERR_CUDA;
 }
 

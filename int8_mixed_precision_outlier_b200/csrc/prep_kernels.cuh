@@ -128,35 +128,52 @@ __global__ void __launch_bounds__(kPrepThreads) detect_partial_kernel(
 
 // ---------------------------------------------------------------------------
 // a4 (prefill): OR the partial flags, write the final bitmask and the
-// ascending outlier index list and its length.  One CTA of 1024 threads;
-// thread i owns words [i*wpt, (i+1)*wpt), so a prefix sum of per-thread
-// counts orders the indices.
+// ascending outlier index list and its length.  One CTA of 1024 threads:
+// the R x Kw partial words are read with 8 loads in flight per thread and
+// OR-ed into shared words; then thread i owns words [i*wpt, (i+1)*wpt), so a
+// prefix sum of per-thread counts orders the indices.
 // ---------------------------------------------------------------------------
 constexpr int kCompactThreads = 1024;
+constexpr int kMaxKw = 65536 / 32;
 
 __global__ void __launch_bounds__(kCompactThreads) compact_kernel(
     const uint32_t* __restrict__ part, int R, int Kw, uint32_t* __restrict__ flags,
     int32_t* __restrict__ idx, int32_t* __restrict__ n_out) {
+  __shared__ uint32_t sw[kMaxKw];
   __shared__ int scratch[33];
   pdl_launch_dependents();
+  for (int w = threadIdx.x; w < Kw; w += kCompactThreads) sw[w] = 0u;
+  __syncthreads();
   pdl_wait();
+  const int items = R * Kw;
+  constexpr int U = 8;
+  for (int base = threadIdx.x; base < items; base += kCompactThreads * U) {
+    uint32_t v[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int e = base + u * kCompactThreads;
+      v[u] = e < items ? __ldg(part + e) : 0u;
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u)
+      if (v[u]) atomicOr(&sw[(base + u * kCompactThreads) % Kw], v[u]);
+  }
+  __syncthreads();
   const int wpt = (Kw + kCompactThreads - 1) / kCompactThreads;
   const int w0 = threadIdx.x * wpt;
   int count = 0;
   for (int i = 0; i < wpt; ++i) {
     const int w = w0 + i;
     if (w >= Kw) break;
-    uint32_t f = 0;
-    for (int r = 0; r < R; ++r) f |= part[(int64_t)r * Kw + w];
-    flags[w] = f;
-    count += __popc(f);
+    flags[w] = sw[w];
+    count += __popc(sw[w]);
   }
   int total;
   int pos = block_exclusive_scan(count, scratch, &total);
   for (int i = 0; i < wpt; ++i) {
     const int w = w0 + i;
     if (w >= Kw) break;
-    uint32_t f = flags[w];
+    uint32_t f = sw[w];
     while (f) {
       const int b = __ffs(f) - 1;
       idx[pos++] = w * 32 + b;
@@ -167,58 +184,60 @@ __global__ void __launch_bounds__(kCompactThreads) compact_kernel(
 }
 
 // ---------------------------------------------------------------------------
-// a2 + a3 + a4 gathers (prefill).  Blocks [0, T): one row of X each -> sx[t],
-// Xq[t, :], Xo[t, 0:Opad) = X[t, idx] (zero past |O|).  Blocks [T, T + nwb):
-// rows of W -> Wo[n, 0:Opad) = W[n, idx].  Opad = |O| rounded up to 64 (one
-// 128-byte fp16 K block of the outlier GEMM).
+// a2 + a3 + a4 gathers (prefill), CTAs of 128 threads.  Blocks
+// [0, gather_ctas): 8 rows of W each -> Wo[n, 0:Opad) = W[n, idx] (zero past
+// |O|), listed first because their scattered loads take longest.  Blocks past
+// those: one row t of X each -> sx[t], Xq[t, :] and Xo[t, 0:Opad) = X[t, idx].
+// The row is read with 4 loads in flight per thread for its absmax, then
+// again (from L1, where this CTA just put it) for its codes.
+// Opad = |O| rounded up to 64 (one 128-byte fp16 K block of the outlier GEMM).
 // ---------------------------------------------------------------------------
-constexpr int kWoRowsPerCta = 16;
+constexpr int kQuantThreads = 128;
+constexpr int kWoRowsPerCta = 8;
+constexpr int kGatherIdxCap = 1024;  // outlier indices staged in shared memory per gather CTA
 
-__global__ void __launch_bounds__(kPrepThreads) quant_gather_kernel(
+__device__ __forceinline__ float block128_max(float v, float* red) {
+  v = warp_max(v);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
+  __syncthreads();
+  const float r = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
+  return r;
+}
+
+__global__ void __launch_bounds__(kQuantThreads) quant_gather_kernel(
     const uint16_t* __restrict__ X, int T, int K, const uint16_t* __restrict__ W, int N,
     const uint32_t* __restrict__ flags, const int32_t* __restrict__ idx,
     const int32_t* __restrict__ n_out, int8_t* __restrict__ Xq, float* __restrict__ sx,
-    uint16_t* __restrict__ Xo, uint16_t* __restrict__ Wo, int ldo) {
-  __shared__ float red[32];
-  pdl_launch_dependents();
+    uint16_t* __restrict__ Xo, uint16_t* __restrict__ Wo, int ldo, int gather_ctas) {
+  __shared__ int32_t si[kGatherIdxCap];
+  __shared__ float red[4];
+  // No early trigger: the GEMM that follows takes a whole SM's shared memory
+  // per CTA, so it launches only as this kernel's CTAs complete.
   pdl_wait();
   const int nO = *n_out;
   const int opad = (nO + 63) & ~63;
-  if (static_cast<int>(blockIdx.x) < T) {
-    const int64_t t = blockIdx.x;
-    const uint4* row = reinterpret_cast<const uint4*>(X + t * K);
-    const uint8_t* fb = reinterpret_cast<const uint8_t*>(flags);
-    const int nchunk = K >> 3;
-    float m = 0.0f;
-    for (int c = threadIdx.x; c < nchunk; c += blockDim.x) m = absmax8(row[c], fb[c], m);
-    const float amax = block_max(m, red);
-    const float s = __fdiv_rn(amax, 127.0f);
-    const float inv = scale_reciprocal(s);
-    if (threadIdx.x == 0) sx[t] = s;
-    uint2* out = reinterpret_cast<uint2*>(Xq + t * K);
-    for (int c = threadIdx.x; c < nchunk; c += blockDim.x) out[c] = quant8(row[c], s, inv, fb[c]);
-    for (int j = threadIdx.x; j < opad; j += blockDim.x)
-      Xo[t * ldo + j] = j < nO ? X[t * K + idx[j]] : uint16_t(0);
-  } else {
-    // Wo rows: every (row, column) pair is an independent item, 4 loads in
-    // flight per thread before their stores.
-    const int64_t n0 = (int64_t)(blockIdx.x - T) * kWoRowsPerCta;
+  if (static_cast<int>(blockIdx.x) < gather_ctas) {
+    const int nstage = nO < kGatherIdxCap ? nO : kGatherIdxCap;
+    for (int j = threadIdx.x; j < nstage; j += blockDim.x) si[j] = idx[j];
+    __syncthreads();
+    const int64_t n0 = static_cast<int64_t>(blockIdx.x) * kWoRowsPerCta;
     const int64_t left = static_cast<int64_t>(N) - n0;
     const int rows = left < kWoRowsPerCta ? static_cast<int>(left) : kWoRowsPerCta;
     const int total = rows * opad;
-    for (int base = threadIdx.x; base < total; base += 4 * blockDim.x) {
-      uint16_t v[4];
+    constexpr int U = 8;
+    for (int base = threadIdx.x; base < total; base += U * blockDim.x) {
+      uint16_t v[U];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
+      for (int u = 0; u < U; ++u) {
         const int e = base + u * blockDim.x;
         v[u] = 0;
         if (e < total) {
           const int rr = e / opad, j = e - rr * opad;
-          if (j < nO) v[u] = __ldg(W + (n0 + rr) * K + idx[j]);
+          if (j < nO) v[u] = __ldg(W + (n0 + rr) * K + (j < kGatherIdxCap ? si[j] : idx[j]));
         }
       }
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
+      for (int u = 0; u < U; ++u) {
         const int e = base + u * blockDim.x;
         if (e < total) {
           const int rr = e / opad, j = e - rr * opad;
@@ -226,7 +245,48 @@ __global__ void __launch_bounds__(kPrepThreads) quant_gather_kernel(
         }
       }
     }
+    return;
   }
+  const int64_t t = blockIdx.x - gather_ctas;
+  const uint4* row = reinterpret_cast<const uint4*>(X + t * K);
+  const uint8_t* fb = reinterpret_cast<const uint8_t*>(flags);
+  uint2* out = reinterpret_cast<uint2*>(Xq + t * K);
+  const int nchunk = K >> 3;
+  constexpr int U = 4;  // loads in flight per thread
+  float m = 0.0f;
+  for (int c0 = threadIdx.x; c0 < nchunk; c0 += kQuantThreads * U) {
+    uint4 v[U];
+    uint32_t f[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int c = c0 + kQuantThreads * u;
+      v[u] = c < nchunk ? __ldg(row + c) : make_uint4(0u, 0u, 0u, 0u);
+      f[u] = c < nchunk ? __ldg(fb + c) : 0xFFu;
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) m = absmax8(v[u], f[u], m);
+  }
+  const float s = __fdiv_rn(block128_max(m, red), 127.0f);
+  const float inv = scale_reciprocal(s);
+  if (threadIdx.x == 0) sx[t] = s;
+  // second pass: the row was just read by this CTA and is still in L1
+  for (int c0 = threadIdx.x; c0 < nchunk; c0 += kQuantThreads * U) {
+    uint4 v[U];
+    uint32_t f[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int c = c0 + kQuantThreads * u;
+      v[u] = c < nchunk ? __ldg(row + c) : make_uint4(0u, 0u, 0u, 0u);
+      f[u] = c < nchunk ? __ldg(fb + c) : 0xFFu;
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int c = c0 + kQuantThreads * u;
+      if (c < nchunk) out[c] = quant8(v[u], s, inv, f[u]);
+    }
+  }
+  for (int j = threadIdx.x; j < opad; j += kQuantThreads)
+    Xo[t * ldo + j] = j < nO ? X[t * K + idx[j]] : uint16_t(0);
 }
 
 // ---------------------------------------------------------------------------
