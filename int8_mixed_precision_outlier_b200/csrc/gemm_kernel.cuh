@@ -30,12 +30,15 @@ constexpr int B_BYTES = BN * BK;              // 32 KiB
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr int THREADS = 192;
 constexpr int TMEM_COLS = 512;                // int32 acc [0, BN) + fp32 yo [BN, 2 BN)
-constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + 256;
+constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + 256 + BN * 4;  // + barriers, + sw of the tile
 
 struct Params {
   int T, N, K;
   int KB;            // int8 k-blocks = ceil(K / BK)
-  int num_m;         // ceil(T / BM)
+  int num_m;         // M tiles: ceil(T / BM), or ceil(T / (2 BM)) for the CTA-pair kernel
+  int num_tiles;     // CTA-pair kernel: num_m * ceil(N / BN)
+  int num_pairs;     // CTA-pair kernel: clusters in the grid
+  int y_tma;         // CTA-pair kernel: 1 = Y written by TMA stores (N % 8 == 0)
   const float* sx;
   const float* sw;
   const int32_t* n_out;
@@ -43,6 +46,69 @@ struct Params {
   int32_t* acc_out;  // optional int32 [T][N]
   uint64_t wait_ns;
 };
+
+// Epilogue of one CTA's 128 x BN output block (rows m0.., columns n0..), run
+// by the 4 epilogue warps (etid = 0..127); warp quadrant q reads TMEM lanes
+// 32q..32q+31 = rows m0+32q+lane:
+//   Y[row, n] = fp16( acc * sx[row] * sw[n] + yo )
+// acc: int32 TMEM columns [0, BN); yo: fp32 columns [BN, 2 BN), read only when
+// there are outlier columns.  The tile's sw values are staged in shared memory
+// (sw_s, BN floats) while the MMAs still run, so that draining TMEM waits on
+// no global load; then it waits (bounded) for `tfull`.
+__device__ __forceinline__ void epilogue_rows(const Params& p, uint32_t tmem_base, int q, int lane, int etid,
+                                              int m0, int n0, uint64_t* tfull, float* sw_s) {
+  for (int j = etid; j < BN; j += 128) sw_s[j] = n0 + j < p.N ? __ldg(p.sw + n0 + j) : 0.0f;
+  named_barrier(1, 128);
+  const int row = m0 + q * 32 + lane;
+  const int nO = *p.n_out;
+  const bool has_o = nO > 0;
+  const float sxr = row < p.T ? p.sx[row] : 0.0f;
+  const bool ok = mbar_wait(tfull, 0, p.wait_ns, kErrTimeoutEpilogue);
+  if (!__all_sync(0xffffffffu, ok)) return;  // warp-uniform before the .sync.aligned loads
+  tc_fence_after();
+  const uint32_t lane_addr = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
+  const bool vec_ok = (p.N % 8) == 0;
+  for (int cc = 0; cc < BN; cc += 32) {
+    if (n0 + cc >= p.N) break;
+    uint32_t ra[32], rb[32];
+    tmem_ld32(lane_addr + cc, ra);
+    if (has_o) tmem_ld32(lane_addr + BN + cc, rb);
+    tmem_ld_wait();
+    if (row < p.T) {
+      const int nbase = n0 + cc;
+      uint32_t packed[16];
+#pragma unroll
+      for (int j = 0; j < 32; j += 2) {
+        float y[2];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const float swn = sw_s[cc + j + h];
+          y[h] = static_cast<float>(static_cast<int32_t>(ra[j + h])) * sxr * swn +
+                 (has_o ? __uint_as_float(rb[j + h]) : 0.0f);
+        }
+        packed[j >> 1] = static_cast<uint32_t>(__half_as_ushort(__float2half_rn(y[0]))) |
+                         (static_cast<uint32_t>(__half_as_ushort(__float2half_rn(y[1]))) << 16);
+      }
+      uint16_t* yrow = p.Y + static_cast<int64_t>(row) * p.N + nbase;
+      if (vec_ok && nbase + 32 <= p.N) {
+        uint4* dst = reinterpret_cast<uint4*>(yrow);
+#pragma unroll
+        for (int v = 0; v < 4; ++v)
+          dst[v] = make_uint4(packed[4 * v], packed[4 * v + 1], packed[4 * v + 2], packed[4 * v + 3]);
+      } else {
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+          if (nbase + j < p.N) yrow[j] = static_cast<uint16_t>(packed[j >> 1] >> ((j & 1) * 16));
+      }
+      if (p.acc_out) {
+        int32_t* arow = p.acc_out + static_cast<int64_t>(row) * p.N + nbase;
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+          if (nbase + j < p.N) arow[j] = static_cast<int32_t>(ra[j]);
+      }
+    }
+  }
+}
 
 __global__ void __launch_bounds__(THREADS, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmap_xq, const __grid_constant__ CUtensorMap tmap_wq,
@@ -163,58 +229,8 @@ __global__ void __launch_bounds__(THREADS, 1)
   } else {
     // ------------------------------------------------------------ epilogue
     pdl_wait();
-    const int q = warp & 3;
-    const int row = m0 + q * 32 + lane;
-    const int nO = *p.n_out;
-    const bool has_o = nO > 0;
-    const float sxr = row < p.T ? p.sx[row] : 0.0f;
-    const bool ok = mbar_wait(tfull, 0, p.wait_ns, kErrTimeoutEpilogue);
-    if (__all_sync(0xffffffffu, ok)) {  // warp-uniform before the .sync.aligned loads
-      tc_fence_after();
-      const uint32_t lane_addr = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
-      const bool vec_ok = (p.N % 8) == 0;
-      for (int cc = 0; cc < BN; cc += 32) {
-        if (n0 + cc >= p.N) break;
-        uint32_t ra[32], rb[32];
-        tmem_ld32(lane_addr + cc, ra);
-        if (has_o) tmem_ld32(lane_addr + BN + cc, rb);
-        tmem_ld_wait();
-        if (row < p.T) {
-          const int nbase = n0 + cc;
-          uint32_t packed[16];
-#pragma unroll
-          for (int j = 0; j < 32; j += 2) {
-            float y[2];
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-              const int n = nbase + j + h;
-              const float swn = n < p.N ? __ldg(p.sw + n) : 0.0f;
-              y[h] = static_cast<float>(static_cast<int32_t>(ra[j + h])) * sxr * swn +
-                     (has_o ? __uint_as_float(rb[j + h]) : 0.0f);
-            }
-            packed[j >> 1] = static_cast<uint32_t>(__half_as_ushort(__float2half_rn(y[0]))) |
-                             (static_cast<uint32_t>(__half_as_ushort(__float2half_rn(y[1]))) << 16);
-          }
-          uint16_t* yrow = p.Y + static_cast<int64_t>(row) * p.N + nbase;
-          if (vec_ok && nbase + 32 <= p.N) {
-            uint4* dst = reinterpret_cast<uint4*>(yrow);
-#pragma unroll
-            for (int v = 0; v < 4; ++v)
-              dst[v] = make_uint4(packed[4 * v], packed[4 * v + 1], packed[4 * v + 2], packed[4 * v + 3]);
-          } else {
-#pragma unroll
-            for (int j = 0; j < 32; ++j)
-              if (nbase + j < p.N) yrow[j] = static_cast<uint16_t>(packed[j >> 1] >> ((j & 1) * 16));
-          }
-          if (p.acc_out) {
-            int32_t* arow = p.acc_out + static_cast<int64_t>(row) * p.N + nbase;
-#pragma unroll
-            for (int j = 0; j < 32; ++j)
-              if (nbase + j < p.N) arow[j] = static_cast<int32_t>(ra[j]);
-          }
-        }
-      }
-    }
+    epilogue_rows(p, tmem_base, warp & 3, lane, static_cast<int>(threadIdx.x) - 64, m0, n0, tfull,
+                  reinterpret_cast<float*>(smem + STAGES * STAGE_BYTES + 256));
   }
 
   // Lane 0 of warps 0 and 1 ran a role loop alone: bring each warp back
@@ -226,6 +242,301 @@ __global__ void __launch_bounds__(THREADS, 1)
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem_base, TMEM_COLS);
+  }
+}
+
+
+// ---------------------------------------------------------------------------
+// CTA-pair kernel for T > BM.  A 2-CTA cluster computes 256 x BN tiles with
+// tcgen05.mma.cta_group::2 (M = 256): CTA r of the pair loads rows
+// m0 + 128 r .. +127 of Xq (A) and rows n0 + 128 r .. +127 of Wq (its half of
+// B), so each SM stages 32 KiB per k-block for its 128 x 256 x 128 share of
+// the products (a single CTA would stage 48 KiB).  The even CTA's thread
+// issues the MMAs; both CTAs' copies complete on the even CTA's `full`
+// barriers and each MMA commit arrives on the `empty` / `tfull` barriers of
+// both CTAs.  TMEM (512 columns in each CTA) holds that CTA's 128 rows: int32
+// acc in [0, BN), fp32 yo in [BN, 2 BN).
+//
+// Persistent: the grid holds as many pairs as fit on the GPU at once (the
+// launch is 2-CTA clusters along x), and pair c takes tiles c, c + pairs, ...
+// The copies of the next tile start while the epilogue drains the current
+// one; its first MMA waits until both CTAs have read their accumulators out
+// (`tempty`, 8 warp arrivals on the even CTA).  The epilogue writes Y through
+// shared memory (two 128 x 64 fp16 staging boxes) and TMA stores, when N is a
+// multiple of 8; otherwise with plain stores.
+// ---------------------------------------------------------------------------
+constexpr int P_STAGES = 6;
+constexpr int P_A_BYTES = BM * BK;                   // 16 KiB: this CTA's 128 rows of Xq
+constexpr int P_B_BYTES = (BN / 2) * BK;             // 16 KiB: this CTA's half of the Wq tile
+constexpr int P_STAGE_BYTES = P_A_BYTES + P_B_BYTES;
+constexpr int P_YCOLS = 64;                          // Y columns per store box (128 bytes)
+constexpr int P_YBUF_BYTES = BM * P_YCOLS * 2;       // 16 KiB
+constexpr int P_SMEM_BYTES = 1024 + P_STAGES * P_STAGE_BYTES + 2 * P_YBUF_BYTES + BN * 4 + 256;
+static_assert(P_SMEM_BYTES <= 232448, "shared memory per CTA");
+
+__device__ __forceinline__ void pair_tile(const Params& p, int tile, uint32_t rank, int* m0, int* n0) {
+  *m0 = (tile % p.num_m) * (2 * BM) + static_cast<int>(rank) * BM;  // this CTA's rows of X / Y
+  *n0 = (tile / p.num_m) * BN;                                      // the pair's columns of Y
+}
+
+// 32 outputs of one row: y = fp16(acc * sxr * sw + yo), packed in pairs.
+__device__ __forceinline__ void dequant32(const uint32_t (&ra)[32], const uint32_t (&rb)[32], bool has_o, float sxr,
+                                          const float* sw32, uint32_t (&packed)[16]) {
+#pragma unroll
+  for (int j = 0; j < 32; j += 2) {
+    float y[2];
+#pragma unroll
+    for (int h = 0; h < 2; ++h)
+      y[h] = static_cast<float>(static_cast<int32_t>(ra[j + h])) * sxr * sw32[j + h] +
+             (has_o ? __uint_as_float(rb[j + h]) : 0.0f);
+    packed[j >> 1] = static_cast<uint32_t>(__half_as_ushort(__float2half_rn(y[0]))) |
+                     (static_cast<uint32_t>(__half_as_ushort(__float2half_rn(y[1]))) << 16);
+  }
+}
+
+__global__ void __launch_bounds__(THREADS, 1)
+    gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_xq, const __grid_constant__ CUtensorMap tmap_wq,
+                     const __grid_constant__ CUtensorMap tmap_xo, const __grid_constant__ CUtensorMap tmap_wo,
+                     const __grid_constant__ CUtensorMap tmap_y, const Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t* ybuf = smem + P_STAGES * P_STAGE_BYTES;                 // [2][128 rows][128 B], 1024-aligned
+  float* sw_s = reinterpret_cast<float*>(ybuf + 2 * P_YBUF_BYTES);  // [BN]
+  uint64_t* full = reinterpret_cast<uint64_t*>(sw_s + BN);          // used in the even CTA
+  uint64_t* empty = full + P_STAGES;
+  uint64_t* tfull = empty + P_STAGES;
+  uint64_t* tempty = tfull + 1;                                     // used in the even CTA
+  uint64_t* done = tempty + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
+
+  const int warp = static_cast<int>(warp_id());
+  const int lane = static_cast<int>(lane_id());
+  const uint32_t rank = cluster_ctarank();  // 0: issues the MMAs
+  const int pair = blockIdx.x >> 1;
+
+  if (warp == 0 && lane == 0) {
+    prefetch_tensormap(&tmap_xq);
+    prefetch_tensormap(&tmap_wq);
+    prefetch_tensormap(&tmap_xo);
+    prefetch_tensormap(&tmap_wo);
+    if (p.y_tma) prefetch_tensormap(&tmap_y);
+    for (int s = 0; s < P_STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(tfull, 1);
+    mbar_init(tempty, 8);  // 4 epilogue warps in each CTA
+    mbar_init(done, 1);
+    fence_barrier_init();
+  }
+  __syncwarp();
+  if (warp == 1) {
+    tmem_alloc_pair(tmem_slot, TMEM_COLS);  // collective with the other CTA's warp 1
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  cluster_sync();  // both CTAs' barriers are initialised before any copy or commit reaches them
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  pdl_launch_dependents();
+
+  auto stage_a = [&](int s) { return smem + s * P_STAGE_BYTES; };
+  auto stage_b = [&](int s) { return smem + s * P_STAGE_BYTES + P_A_BYTES; };
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer (both CTAs)
+    if (lane == 0 && pair < p.num_tiles) {
+      const bool lead = rank == 0;
+      const int KB = p.KB;
+      auto full_of = [&](int s) { return map_shared_rank(&full[s], 0); };
+      int m0, n0;
+      pair_tile(p, pair, rank, &m0, &n0);
+      // Wq does not depend on the preceding kernels: the first tile's first
+      // stages are requested before waiting for them.  The even CTA arms its
+      // barrier for both CTAs' bytes; the odd CTA's copies may land before
+      // that (the phase still waits for the arrival).
+      const int pre = KB < P_STAGES ? KB : P_STAGES;
+      for (int i = 0; i < pre; ++i) {
+        if (lead) mbar_arrive_expect_tx(&full[i], 2 * P_STAGE_BYTES);
+        tma_load_2d_pair(stage_b(i), &tmap_wq, full_of(i), i * BK, n0 + static_cast<int>(rank) * (BN / 2));
+      }
+      pdl_wait();
+      for (int i = 0; i < pre; ++i) tma_load_2d_pair(stage_a(i), &tmap_xq, full_of(i), i * BK, m0);
+      const int total = KB + (*p.n_out + 63) / 64;
+      int it = pre;  // k-blocks issued so far, over all tiles: stage it % P_STAGES
+      int kb = pre;
+      bool ok = true;
+      for (int tile = pair; ok && tile < p.num_tiles; tile += p.num_pairs, kb = 0) {
+        pair_tile(p, tile, rank, &m0, &n0);
+        const int nb0 = n0 + static_cast<int>(rank) * (BN / 2);
+        for (; kb < total; ++kb, ++it) {
+          const int s = it % P_STAGES;
+          if (it >= P_STAGES &&
+              !mbar_wait(&empty[s], ((it / P_STAGES) & 1) ^ 1, p.wait_ns, kErrTimeoutProducer)) {
+            ok = false;
+            break;
+          }
+          if (lead) mbar_arrive_expect_tx(&full[s], 2 * P_STAGE_BYTES);
+          if (kb < KB) {
+            tma_load_2d_pair(stage_a(s), &tmap_xq, full_of(s), kb * BK, m0);
+            tma_load_2d_pair(stage_b(s), &tmap_wq, full_of(s), kb * BK, nb0);
+          } else {
+            const int jb = kb - KB;
+            tma_load_2d_pair(stage_a(s), &tmap_xo, full_of(s), jb * 64, m0);
+            tma_load_2d_pair(stage_b(s), &tmap_wo, full_of(s), jb * 64, nb0);
+          }
+        }
+      }
+      // Every copy has landed once the MMAs that read it completed: the
+      // `done` commit covers that on the normal path.
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer (even CTA)
+    if (lane == 0 && rank == 0) {
+      pdl_wait();
+      const int total = p.KB + (*p.n_out + 63) / 64;
+      constexpr uint32_t idesc_i = idesc_i8_s32(2 * BM, BN);
+      constexpr uint32_t idesc_h = idesc_f16_f32(2 * BM, BN);
+      const uint32_t d_acc = tmem_base;
+      const uint32_t d_yo = tmem_base + BN;
+      bool ok = true;
+      int it = 0, tc = 0;
+      for (int tile = pair; ok && tile < p.num_tiles; tile += p.num_pairs, ++tc) {
+        if (tc > 0) {  // both CTAs have drained the previous tile's accumulators
+          ok = mbar_wait_cluster(tempty, (tc - 1) & 1, p.wait_ns, kErrTimeoutMma);
+          if (!ok) break;
+        }
+        tc_fence_after();
+        for (int kb = 0; kb < total; ++kb, ++it) {
+          const int s = it % P_STAGES;
+          ok = mbar_wait(&full[s], (it / P_STAGES) & 1, p.wait_ns, kErrTimeoutMma);
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t a0 = smem_addr(stage_a(s));
+          const uint32_t b0 = smem_addr(stage_b(s));
+          if (kb < p.KB) {
+#pragma unroll
+            for (int k = 0; k < BK / 32; ++k)
+              mma_i8_pair(d_acc, make_sdesc_k_sw128(a0 + k * 32), make_sdesc_k_sw128(b0 + k * 32), idesc_i,
+                          (kb > 0 || k > 0) ? 1u : 0u);
+          } else {
+#pragma unroll
+            for (int k = 0; k < BK / 32; ++k)
+              mma_f16_pair(d_yo, make_sdesc_k_sw128(a0 + k * 32), make_sdesc_k_sw128(b0 + k * 32), idesc_h,
+                           (kb > p.KB || k > 0) ? 1u : 0u);
+          }
+          mma_commit_pair(&empty[s], 0x3);
+        }
+        if (ok) mma_commit_pair(tfull, 0x3);
+      }
+      mma_commit_pair(done, 0x3);
+    }
+    // Both CTAs: the pair's MMAs are complete before TMEM is released.
+    if (lane == 0) mbar_wait(done, 0, p.wait_ns, kErrTimeoutMma);
+  } else {
+    // ------------------------------------------------------------ epilogue (both CTAs)
+    const int q = warp & 3;         // TMEM lane quadrant of this warp
+    const int etid = static_cast<int>(threadIdx.x) - 64;
+    const int r_loc = q * 32 + lane;  // row within this CTA's 128
+    pdl_wait();
+    const bool has_o = *p.n_out > 0;
+    const uint32_t tempty_lead = map_shared_rank(tempty, 0);
+    const uint32_t lane_addr = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
+    const bool vec_ok = (p.N % 8) == 0;
+    int tc = 0, stores = 0;
+    for (int tile = pair; tile < p.num_tiles; tile += p.num_pairs, ++tc) {
+      int m0, n0;
+      pair_tile(p, tile, rank, &m0, &n0);
+      named_barrier(1, 128);  // every thread is past the previous tile's reads of sw_s
+      for (int j = etid; j < BN; j += 128) sw_s[j] = n0 + j < p.N ? __ldg(p.sw + n0 + j) : 0.0f;
+      named_barrier(1, 128);
+      const int row = m0 + r_loc;
+      const float sxr = row < p.T ? p.sx[row] : 0.0f;
+      const bool okw = mbar_wait(tfull, tc & 1, p.wait_ns, kErrTimeoutEpilogue);
+      if (!named_barrier_and(2, 128, okw)) break;  // all 128 threads leave together
+      tc_fence_after();
+      for (int g = 0; g < BN / P_YCOLS; ++g) {
+        const bool active = n0 + g * P_YCOLS < p.N;        // uniform
+        const bool staged = p.y_tma && active && m0 < p.T;  // uniform: a store with rows to write
+        uint8_t* yb = ybuf + (stores & 1) * P_YBUF_BYTES;
+        if (staged) {
+          // The store that last read this staging box has finished with it.
+          if (etid == 0) bulk_wait_group_read<1>();
+          named_barrier(1, 128);
+        }
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int c0 = g * P_YCOLS + h * 32;  // first column of these 32
+          uint32_t ra[32], rb[32];
+          tmem_ld32(lane_addr + c0, ra);
+          if (has_o) tmem_ld32(lane_addr + BN + c0, rb);
+          tmem_ld_wait();
+          if (g == BN / P_YCOLS - 1 && h == 1) {
+            // This warp has read all of its accumulators: the next tile's
+            // MMAs may overwrite them.
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(tempty_lead);
+          }
+          if (!active) continue;
+          uint32_t packed[16];
+          dequant32(ra, rb, has_o, sxr, sw_s + c0, packed);
+          if (staged) {
+            // 128-byte swizzle, as the store's tensor map expects: 16-byte
+            // chunk c of a row sits at chunk c ^ (row % 8).
+            uint8_t* rowp = yb + r_loc * 128;
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+              const int c = h * 4 + v;
+              *reinterpret_cast<uint4*>(rowp + ((c ^ (r_loc & 7)) << 4)) =
+                  make_uint4(packed[4 * v], packed[4 * v + 1], packed[4 * v + 2], packed[4 * v + 3]);
+            }
+          } else if (!p.y_tma && row < p.T) {
+            const int nbase = n0 + c0;
+            uint16_t* yrow = p.Y + static_cast<int64_t>(row) * p.N + nbase;
+            if (vec_ok && nbase + 32 <= p.N) {
+              uint4* dst = reinterpret_cast<uint4*>(yrow);
+#pragma unroll
+              for (int v = 0; v < 4; ++v)
+                dst[v] = make_uint4(packed[4 * v], packed[4 * v + 1], packed[4 * v + 2], packed[4 * v + 3]);
+            } else {
+#pragma unroll
+              for (int j = 0; j < 32; ++j)
+                if (nbase + j < p.N) yrow[j] = static_cast<uint16_t>(packed[j >> 1] >> ((j & 1) * 16));
+            }
+          }
+          if (p.acc_out && row < p.T) {
+            const int nbase = n0 + c0;
+            int32_t* arow = p.acc_out + static_cast<int64_t>(row) * p.N + nbase;
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              if (nbase + j < p.N) arow[j] = static_cast<int32_t>(ra[j]);
+          }
+        }
+        if (staged) {
+          fence_proxy_async_shared();  // the staging writes, before the async-proxy store reads them
+          named_barrier(1, 128);
+          if (etid == 0) {
+            tma_store_2d(&tmap_y, yb, n0 + g * P_YCOLS, m0);
+            bulk_commit_group();
+          }
+          ++stores;
+        }
+      }
+    }
+    if (etid == 0) bulk_wait_group<0>();  // Y is written before the CTA ends
+  }
+
+  __syncwarp();
+  tc_fence_before();
+  // Neither CTA leaves while the other may still signal its barriers or, after
+  // a timeout, copies of the pair may still be landing.
+  if (threadIdx.x == 0 && ld_error_word() != 0) sleep_ns_bounded(20000);
+  cluster_sync();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, TMEM_COLS);
   }
 }
 

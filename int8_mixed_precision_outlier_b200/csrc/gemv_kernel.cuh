@@ -216,6 +216,12 @@ __global__ void __launch_bounds__(THREADS, 1)
         mbar_arrive_expect_tx(&full[i], STAGE_BYTES);
         tma_load_2d_hint(stage_a(i), &tmap_w, &full[i], (u % p.KB) * BK, (u / p.KB) * BM, pol);
       }
+      // The rest of this CTA's weight range goes to L2 now, so that HBM keeps
+      // streaming while the ring is full and the activation codes are made.
+      for (int i = pre; i < n_units; ++i) {
+        const int u = u0 + i;
+        tma_prefetch_l2_2d(&tmap_w, (u % p.KB) * BK, (u / p.KB) * BM);
+      }
       pdl_wait();
       for (int i = 0; i < pre; ++i) {
         const int u = u0 + i;

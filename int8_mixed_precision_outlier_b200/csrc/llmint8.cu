@@ -37,10 +37,11 @@ struct DeviceInfo {
   std::once_flag once;
   int status = LLMINT8_OK;
   int num_sms = 0;
+  int max_pairs = 0;  // 2-CTA clusters of gemm_pair_kernel resident at once
 };
 DeviceInfo g_dev[kMaxDevices];
 
-int device_info(int* num_sms) {
+int device_info(int* num_sms, int* max_pairs = nullptr) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return LLMINT8_ERR_CUDA;
   if (dev < 0 || dev >= kMaxDevices) return LLMINT8_ERR_CUDA;
@@ -59,6 +60,8 @@ int device_info(int* num_sms) {
     }
     if (cudaFuncSetAttribute(gemm::gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              gemm::SMEM_BYTES) != cudaSuccess ||
+        cudaFuncSetAttribute(gemm::gemm_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             gemm::P_SMEM_BYTES) != cudaSuccess ||
         cudaFuncSetAttribute(gemv::gemv_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              gemv::SMEM_BYTES) != cudaSuccess ||
         cudaFuncSetAttribute(gemv::gemv_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -73,8 +76,28 @@ int device_info(int* num_sms) {
       return;
     }
     d.num_sms = sms;
+    // How many pairs the persistent GEMM can keep resident (GPCs with an odd
+    // number of usable SMs leave one idle).
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * (sms / 2));
+    cfg.blockDim = dim3(gemm::THREADS);
+    cfg.dynamicSmemBytes = gemm::P_SMEM_BYTES;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int clusters = 0;
+    if (cudaOccupancyMaxActiveClusters(&clusters, gemm::gemm_pair_kernel, &cfg) != cudaSuccess || clusters < 1) {
+      cudaGetLastError();
+      clusters = sms / 2;
+    }
+    d.max_pairs = clusters;
   });
   if (num_sms) *num_sms = d.num_sms;
+  if (max_pairs) *max_pairs = d.max_pairs;
   return d.status;
 }
 
@@ -284,8 +307,8 @@ int matmul_impl(const void* Xv, int64_t T, int64_t K, const int8_t* Wq, const fl
       (reinterpret_cast<uintptr_t>(ins.sx) & 3u) || (reinterpret_cast<uintptr_t>(ins.idx) & 3u) ||
       (reinterpret_cast<uintptr_t>(ins.n) & 3u))
     return LLMINT8_ERR_ALIGNMENT;
-  int num_sms = 0;
-  rc = device_info(&num_sms);
+  int num_sms = 0, max_pairs = 0;
+  rc = device_info(&num_sms, &max_pairs);
   if (rc != LLMINT8_OK) return rc;
 
   cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -345,7 +368,9 @@ int matmul_impl(const void* Xv, int64_t T, int64_t K, const int8_t* Wq, const fl
   p.N = n;
   p.K = k;
   p.KB = (k + gemm::BK - 1) / gemm::BK;
-  p.num_m = (t + gemm::BM - 1) / gemm::BM;
+  // More than one 128-row tile of tokens: CTA pairs, 256 rows per tile.
+  const bool pair = t > gemm::BM;
+  p.num_m = pair ? (t + 2 * gemm::BM - 1) / (2 * gemm::BM) : (t + gemm::BM - 1) / gemm::BM;
   p.sx = out.sx;
   p.sw = Wscale;
   p.n_out = out.n_out;
@@ -353,20 +378,30 @@ int matmul_impl(const void* Xv, int64_t T, int64_t K, const int8_t* Wq, const fl
   p.acc_out = acc_out;
   p.wait_ns = wait_ns;
   const int num_n = (n + gemm::BN - 1) / gemm::BN;
-  CUtensorMap txq, twq, txo, two;
+  p.num_tiles = p.num_m * num_n;
+  p.num_pairs = pair ? (p.num_tiles < max_pairs ? p.num_tiles : max_pairs) : 0;
+  p.y_tma = (pair && n % 8 == 0) ? 1 : 0;
+  CUtensorMap txq, twq, txo, two, ty;
+  std::memset(&ty, 0, sizeof(ty));
+  if (p.y_tma && !encode_2d(&ty, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, Y, N, T, 2ull * N, gemm::P_YCOLS, gemm::BM))
+    return LLMINT8_ERR_CUDA;
   const uint16_t* xo = reinterpret_cast<const uint16_t*>(ws + L.xo);
   const uint16_t* wo = reinterpret_cast<const uint16_t*>(ws + L.wo);
   if (!encode_2d(&txq, CU_TENSOR_MAP_DATA_TYPE_UINT8, out.xq, K, T, K, gemm::BK, gemm::BM) ||
-      !encode_2d(&twq, CU_TENSOR_MAP_DATA_TYPE_UINT8, Wq, K, N, K, gemm::BK, gemm::BN) ||
+      !encode_2d(&twq, CU_TENSOR_MAP_DATA_TYPE_UINT8, Wq, K, N, K, gemm::BK, pair ? gemm::BN / 2 : gemm::BN) ||
       !encode_2d(&txo, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, xo, L.ldo, T, 2ull * L.ldo, 64, gemm::BM) ||
-      !encode_2d(&two, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, wo, L.ldo, N, 2ull * L.ldo, 64, gemm::BN))
+      !encode_2d(&two, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, wo, L.ldo, N, 2ull * L.ldo, 64,
+                 pair ? gemm::BN / 2 : gemm::BN))
     return LLMINT8_ERR_CUDA;
   rc = launch_prep(L, X, t, k, W, n, threshold, ws, out, st);
   if (rc != LLMINT8_OK) return rc;
   if (ev_begin && cudaEventRecord(ev_begin, st) != cudaSuccess) return LLMINT8_ERR_CUDA;
   for (int r = 0; r < repeat; ++r) {
-    cudaError_t e = launch(gemm::gemm_kernel, dim3(p.num_m * num_n), dim3(gemm::THREADS), gemm::SMEM_BYTES,
-                           st, true, txq, twq, txo, two, p);
+    const cudaError_t e =
+        pair ? launch_ex(gemm::gemm_pair_kernel, dim3(2 * p.num_pairs), dim3(gemm::THREADS),
+                         gemm::P_SMEM_BYTES, st, true, 2, txq, twq, txo, two, ty, p)
+             : launch(gemm::gemm_kernel, dim3(p.num_m * num_n), dim3(gemm::THREADS), gemm::SMEM_BYTES, st, true,
+                      txq, twq, txo, two, p);
     if (e != cudaSuccess) return LLMINT8_ERR_CUDA;
   }
   if (ev_end && cudaEventRecord(ev_end, st) != cudaSuccess) return LLMINT8_ERR_CUDA;
