@@ -164,7 +164,7 @@ LLMINT8_API int llmint8_detect_quantize(const void* X, int64_t T, int64_t K, flo
  * all device memory through its own pool (a library may not take memory behind
  * its back) or a latency-critical loop where an allocation could stall the
  * device or fail mid-run.  Scratch comes from one fixed array in device memory
- * per GPU that loads the library (5 MiB, kept until the process exits).
+ * per GPU that loads the library (1 MiB, kept until the process exits).
  *   Limits: 1 <= T <= 16, 16 <= K <= 16384, K % 16 == 0, 1 <= N <= 65536;
  *   larger sizes return LLMINT8_ERR_INVALID_ARG and launch nothing.
  *   The first call on a device looks up that device's array address (a

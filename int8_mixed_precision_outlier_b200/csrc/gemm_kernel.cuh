@@ -36,9 +36,10 @@ struct Params {
   int T, N, K;
   int KB;            // int8 k-blocks = ceil(K / BK)
   int num_m;         // M tiles: ceil(T / BM), or ceil(T / (2 BM)) for the CTA-pair kernel
-  int num_tiles;     // CTA-pair kernel: num_m * ceil(N / BN)
+  int num_tiles;     // CTA-pair kernel: num_m * ceil(N / bn)
   int num_pairs;     // CTA-pair kernel: clusters in the grid
   int y_tma;         // CTA-pair kernel: 1 = Y written by TMA stores (N % 8 == 0)
+  int bn;            // CTA-pair kernel: tile columns (128, 192 or 256)
   const float* sx;
   const float* sw;
   const int32_t* n_out;
@@ -247,25 +248,31 @@ __global__ void __launch_bounds__(THREADS, 1)
 
 
 // ---------------------------------------------------------------------------
-// CTA-pair kernel for T > BM.  A 2-CTA cluster computes 256 x BN tiles with
-// tcgen05.mma.cta_group::2 (M = 256): CTA r of the pair loads rows
-// m0 + 128 r .. +127 of Xq (A) and rows n0 + 128 r .. +127 of Wq (its half of
-// B), so each SM stages 32 KiB per k-block for its 128 x 256 x 128 share of
-// the products (a single CTA would stage 48 KiB).  The even CTA's thread
+// CTA-pair kernel for T > BM.  A 2-CTA cluster computes 256 x bn tiles with
+// tcgen05.mma.cta_group::2 (M = 256, N = bn, bn = 128, 192 or 256, chosen by
+// the host so that the tiles spread evenly over the resident pairs): CTA r of
+// the pair loads rows m0 + 128 r .. +127 of Xq (A) and rows
+// n0 + bn/2 r .. + bn/2 - 1 of Wq (its half of B), so at bn = 256 each SM
+// stages 32 KiB per k-block for its 128 x 256 x 128 share of the products (a
+// single CTA would stage 48 KiB).  The even CTA's thread
 // issues the MMAs; both CTAs' copies complete on the even CTA's `full`
 // barriers and each MMA commit arrives on the `empty` / `tfull` barriers of
 // both CTAs.  TMEM (512 columns in each CTA) holds that CTA's 128 rows: int32
-// acc in [0, BN), fp32 yo in [BN, 2 BN).
+// acc in [0, bn), fp32 yo in [bn, 2 bn).
 //
 // Persistent: the grid holds as many pairs as fit on the GPU at once (the
 // launch is 2-CTA clusters along x), and pair c takes tiles c, c + pairs, ...
 // The copies of the next tile start while the epilogue drains the current
 // one; its first MMA waits until both CTAs have read their accumulators out
-// (`tempty`, 8 warp arrivals on the even CTA).  The epilogue writes Y through
-// shared memory (two 128 x 64 fp16 staging boxes) and TMA stores, when N is a
-// multiple of 8; otherwise with plain stores.
+// (`tempty`, one arrival per epilogue warp of both CTAs, on the even CTA).
+// The epilogue runs in two sets of 4 warps; set s drains the 64-column groups
+// g = s, s + 2, ... of the tile 32 columns at a time and writes Y through its
+// own shared-memory staging box (128 x 64 fp16) and a TMA store when N is a
+// multiple of 8, otherwise with plain stores.
 // ---------------------------------------------------------------------------
 constexpr int P_STAGES = 6;
+constexpr int P_THREADS = 320;                       // warp 0 TMA, warp 1 MMA, warps 2-9 epilogue
+constexpr int P_EPI_WARPS = 8;                       // two sets of 4: one warp per TMEM lane quadrant each
 constexpr int P_A_BYTES = BM * BK;                   // 16 KiB: this CTA's 128 rows of Xq
 constexpr int P_B_BYTES = (BN / 2) * BK;             // 16 KiB: this CTA's half of the Wq tile
 constexpr int P_STAGE_BYTES = P_A_BYTES + P_B_BYTES;
@@ -276,7 +283,7 @@ static_assert(P_SMEM_BYTES <= 232448, "shared memory per CTA");
 
 __device__ __forceinline__ void pair_tile(const Params& p, int tile, uint32_t rank, int* m0, int* n0) {
   *m0 = (tile % p.num_m) * (2 * BM) + static_cast<int>(rank) * BM;  // this CTA's rows of X / Y
-  *n0 = (tile / p.num_m) * BN;                                      // the pair's columns of Y
+  *n0 = (tile / p.num_m) * p.bn;                                    // the pair's columns of Y
 }
 
 // 32 outputs of one row: y = fp16(acc * sxr * sw + yo), packed in pairs.
@@ -289,12 +296,12 @@ __device__ __forceinline__ void dequant32(const uint32_t (&ra)[32], const uint32
     for (int h = 0; h < 2; ++h)
       y[h] = static_cast<float>(static_cast<int32_t>(ra[j + h])) * sxr * sw32[j + h] +
              (has_o ? __uint_as_float(rb[j + h]) : 0.0f);
-    packed[j >> 1] = static_cast<uint32_t>(__half_as_ushort(__float2half_rn(y[0]))) |
-                     (static_cast<uint32_t>(__half_as_ushort(__float2half_rn(y[1]))) << 16);
+    const __half2 h2 = __floats2half2_rn(y[0], y[1]);  // y[0] in the low half
+    packed[j >> 1] = *reinterpret_cast<const uint32_t*>(&h2);
   }
 }
 
-__global__ void __launch_bounds__(THREADS, 1)
+__global__ void __launch_bounds__(P_THREADS, 1)
     gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_xq, const __grid_constant__ CUtensorMap tmap_wq,
                      const __grid_constant__ CUtensorMap tmap_xo, const __grid_constant__ CUtensorMap tmap_wo,
                      const __grid_constant__ CUtensorMap tmap_y, const Params p) {
@@ -326,7 +333,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       mbar_init(&empty[s], 1);
     }
     mbar_init(tfull, 1);
-    mbar_init(tempty, 8);  // 4 epilogue warps in each CTA
+    mbar_init(tempty, 2 * P_EPI_WARPS);  // every epilogue warp of both CTAs
     mbar_init(done, 1);
     fence_barrier_init();
   }
@@ -357,9 +364,10 @@ __global__ void __launch_bounds__(THREADS, 1)
       // barrier for both CTAs' bytes; the odd CTA's copies may land before
       // that (the phase still waits for the arrival).
       const int pre = KB < P_STAGES ? KB : P_STAGES;
+      const uint32_t stage_tx = 2u * static_cast<uint32_t>(P_A_BYTES + (p.bn / 2) * BK);  // both CTAs
       for (int i = 0; i < pre; ++i) {
-        if (lead) mbar_arrive_expect_tx(&full[i], 2 * P_STAGE_BYTES);
-        tma_load_2d_pair(stage_b(i), &tmap_wq, full_of(i), i * BK, n0 + static_cast<int>(rank) * (BN / 2));
+        if (lead) mbar_arrive_expect_tx(&full[i], stage_tx);
+        tma_load_2d_pair(stage_b(i), &tmap_wq, full_of(i), i * BK, n0 + static_cast<int>(rank) * (p.bn / 2));
       }
       pdl_wait();
       for (int i = 0; i < pre; ++i) tma_load_2d_pair(stage_a(i), &tmap_xq, full_of(i), i * BK, m0);
@@ -369,7 +377,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       bool ok = true;
       for (int tile = pair; ok && tile < p.num_tiles; tile += p.num_pairs, kb = 0) {
         pair_tile(p, tile, rank, &m0, &n0);
-        const int nb0 = n0 + static_cast<int>(rank) * (BN / 2);
+        const int nb0 = n0 + static_cast<int>(rank) * (p.bn / 2);
         for (; kb < total; ++kb, ++it) {
           const int s = it % P_STAGES;
           if (it >= P_STAGES &&
@@ -377,7 +385,7 @@ __global__ void __launch_bounds__(THREADS, 1)
             ok = false;
             break;
           }
-          if (lead) mbar_arrive_expect_tx(&full[s], 2 * P_STAGE_BYTES);
+          if (lead) mbar_arrive_expect_tx(&full[s], stage_tx);
           if (kb < KB) {
             tma_load_2d_pair(stage_a(s), &tmap_xq, full_of(s), kb * BK, m0);
             tma_load_2d_pair(stage_b(s), &tmap_wq, full_of(s), kb * BK, nb0);
@@ -396,10 +404,10 @@ __global__ void __launch_bounds__(THREADS, 1)
     if (lane == 0 && rank == 0) {
       pdl_wait();
       const int total = p.KB + (*p.n_out + 63) / 64;
-      constexpr uint32_t idesc_i = idesc_i8_s32(2 * BM, BN);
-      constexpr uint32_t idesc_h = idesc_f16_f32(2 * BM, BN);
+      const uint32_t idesc_i = idesc_i8_s32(2 * BM, p.bn);
+      const uint32_t idesc_h = idesc_f16_f32(2 * BM, p.bn);
       const uint32_t d_acc = tmem_base;
-      const uint32_t d_yo = tmem_base + BN;
+      const uint32_t d_yo = tmem_base + static_cast<uint32_t>(p.bn);
       bool ok = true;
       int it = 0, tc = 0;
       for (int tile = pair; ok && tile < p.num_tiles; tile += p.num_pairs, ++tc) {
@@ -436,50 +444,67 @@ __global__ void __launch_bounds__(THREADS, 1)
     if (lane == 0) mbar_wait(done, 0, p.wait_ns, kErrTimeoutMma);
   } else {
     // ------------------------------------------------------------ epilogue (both CTAs)
-    const int q = warp & 3;         // TMEM lane quadrant of this warp
-    const int etid = static_cast<int>(threadIdx.x) - 64;
-    const int r_loc = q * 32 + lane;  // row within this CTA's 128
+    const int set = (warp - 2) >> 2;                           // 0 or 1
+    const int q = warp & 3;                                    // TMEM lane quadrant of this warp
+    const int etid = static_cast<int>(threadIdx.x) - 64;       // 0..255
+    const int stid = etid - 128 * set;                         // 0..127 within the set
+    const uint32_t set_bar = 1u + 2u * static_cast<uint32_t>(set);  // named barriers 1 / 3
+    const int r_loc = q * 32 + lane;                           // row within this CTA's 128
+    uint8_t* yb = ybuf + set * P_YBUF_BYTES;                   // this set's staging box
     pdl_wait();
     const bool has_o = *p.n_out > 0;
     const uint32_t tempty_lead = map_shared_rank(tempty, 0);
     const uint32_t lane_addr = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
+    const uint32_t yo_col = static_cast<uint32_t>(p.bn);
     const bool vec_ok = (p.N % 8) == 0;
-    int tc = 0, stores = 0;
+    const int groups = p.bn / P_YCOLS;
+    int tc = 0;
     for (int tile = pair; tile < p.num_tiles; tile += p.num_pairs, ++tc) {
       int m0, n0;
       pair_tile(p, tile, rank, &m0, &n0);
-      named_barrier(1, 128);  // every thread is past the previous tile's reads of sw_s
-      for (int j = etid; j < BN; j += 128) sw_s[j] = n0 + j < p.N ? __ldg(p.sw + n0 + j) : 0.0f;
-      named_barrier(1, 128);
+      named_barrier(5, 2 * 128);  // both sets are past the previous tile's reads of sw_s
+      for (int j = etid; j < p.bn; j += 2 * 128) sw_s[j] = n0 + j < p.N ? __ldg(p.sw + n0 + j) : 0.0f;
+      named_barrier(5, 2 * 128);
       const int row = m0 + r_loc;
       const float sxr = row < p.T ? p.sx[row] : 0.0f;
       const bool okw = mbar_wait(tfull, tc & 1, p.wait_ns, kErrTimeoutEpilogue);
-      if (!named_barrier_and(2, 128, okw)) break;  // all 128 threads leave together
+      if (!named_barrier_and(2, 2 * 128, okw)) break;  // all 256 epilogue threads leave together
       tc_fence_after();
-      for (int g = 0; g < BN / P_YCOLS; ++g) {
+      for (int g = set; g < groups; g += 2) {
+        const bool last_group = g + 2 >= groups;
         const bool active = n0 + g * P_YCOLS < p.N;        // uniform
         const bool staged = p.y_tma && active && m0 < p.T;  // uniform: a store with rows to write
-        uint8_t* yb = ybuf + (stores & 1) * P_YBUF_BYTES;
-        if (staged) {
-          // The store that last read this staging box has finished with it.
-          if (etid == 0) bulk_wait_group_read<1>();
-          named_barrier(1, 128);
+        // The group's 64 columns of both accumulators go to registers first,
+        // so that after the last group TMEM is released before any wait on a
+        // store.
+        uint32_t ra0[32], rb0[32], ra1[32], rb1[32];
+        const uint32_t cg = static_cast<uint32_t>(g * P_YCOLS);
+        tmem_ld32(lane_addr + cg, ra0);
+        tmem_ld32(lane_addr + cg + 32, ra1);
+        if (has_o) {
+          tmem_ld32(lane_addr + yo_col + cg, rb0);
+          tmem_ld32(lane_addr + yo_col + cg + 32, rb1);
         }
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const int c0 = g * P_YCOLS + h * 32;  // first column of these 32
-          uint32_t ra[32], rb[32];
-          tmem_ld32(lane_addr + c0, ra);
-          if (has_o) tmem_ld32(lane_addr + BN + c0, rb);
-          tmem_ld_wait();
-          if (g == BN / P_YCOLS - 1 && h == 1) {
-            // This warp has read all of its accumulators: the next tile's
-            // MMAs may overwrite them.
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive_cluster(tempty_lead);
-          }
-          if (!active) continue;
+        tmem_ld_wait();
+        tmem_regs_ready(ra0);
+        tmem_regs_ready(ra1);
+        tmem_regs_ready(rb0);
+        tmem_regs_ready(rb1);
+        if (last_group) {
+          // This warp has read all of its accumulators: the next tile's MMAs
+          // may overwrite them.
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive_cluster(tempty_lead);
+        }
+        if (!active) continue;
+        if (staged) {
+          if (stid == 0) bulk_wait_group_read<0>();  // this set's previous store is done with the box
+          named_barrier(set_bar, 128);
+        }
+        // 32 columns starting at c0 = g * 64 + 32 h.
+        auto half = [&](int h, const uint32_t (&ra)[32], const uint32_t (&rb)[32]) {
+          const int c0 = g * P_YCOLS + h * 32;
           uint32_t packed[16];
           dequant32(ra, rb, has_o, sxr, sw_s + c0, packed);
           if (staged) {
@@ -513,19 +538,20 @@ __global__ void __launch_bounds__(THREADS, 1)
             for (int j = 0; j < 32; ++j)
               if (nbase + j < p.N) arow[j] = static_cast<int32_t>(ra[j]);
           }
-        }
+        };
+        half(0, ra0, rb0);
+        half(1, ra1, rb1);
         if (staged) {
           fence_proxy_async_shared();  // the staging writes, before the async-proxy store reads them
-          named_barrier(1, 128);
-          if (etid == 0) {
+          named_barrier(set_bar, 128);
+          if (stid == 0) {
             tma_store_2d(&tmap_y, yb, n0 + g * P_YCOLS, m0);
             bulk_commit_group();
           }
-          ++stores;
         }
       }
     }
-    if (etid == 0) bulk_wait_group<0>();  // Y is written before the CTA ends
+    if (stid == 0) bulk_wait_group<0>();  // Y is written before the CTA ends
   }
 
   __syncwarp();

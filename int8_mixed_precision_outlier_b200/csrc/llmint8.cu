@@ -71,7 +71,21 @@ int device_info(int* num_sms, int* max_pairs = nullptr) {
         cudaFuncSetAttribute(gemv::gemv_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              gemv::SMEM_BYTES) != cudaSuccess ||
         cudaFuncSetAttribute(gemv::gemv_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             gemv::SMEM_BYTES) != cudaSuccess) {
+                             gemv::SMEM_BYTES) != cudaSuccess ||
+        // The decode prep kernel runs next to GEMV CTAs (its own call's, which
+        // launch early, and the previous call's): with the largest shared
+        // memory carveout on its SMs, a GEMV CTA fits beside it instead of
+        // waiting for it to finish.
+        cudaFuncSetAttribute(decode_prep_kernel<1>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             cudaSharedmemCarveoutMaxShared) != cudaSuccess ||
+        cudaFuncSetAttribute(decode_prep_kernel<2>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             cudaSharedmemCarveoutMaxShared) != cudaSuccess ||
+        cudaFuncSetAttribute(decode_prep_kernel<4>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             cudaSharedmemCarveoutMaxShared) != cudaSuccess ||
+        cudaFuncSetAttribute(decode_prep_kernel<8>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             cudaSharedmemCarveoutMaxShared) != cudaSuccess ||
+        cudaFuncSetAttribute(decode_prep_kernel<16>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             cudaSharedmemCarveoutMaxShared) != cudaSuccess) {
       d.status = LLMINT8_ERR_CUDA;
       return;
     }
@@ -80,7 +94,7 @@ int device_info(int* num_sms, int* max_pairs = nullptr) {
     // number of usable SMs leave one idle).
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(2 * (sms / 2));
-    cfg.blockDim = dim3(gemm::THREADS);
+    cfg.blockDim = dim3(gemm::P_THREADS);
     cfg.dynamicSmemBytes = gemm::P_SMEM_BYTES;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -137,14 +151,30 @@ bool encode_2d(CUtensorMap* map, CUtensorMapDataType dt, const void* base, uint6
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Int8 matrix [rows][K] (K % 128 == 0) seen as 3-D: 128 bytes of a k-block,
+// row, k-block; a box of `box_rows` rows x `kpb` k-blocks lands as kpb
+// consecutive 128-byte-swizzled tiles of box_rows x 128 bytes, and reads
+// kpb * 128 contiguous bytes of every row.
+bool encode_kblocks_3d(CUtensorMap* map, const void* base, uint64_t rows, uint64_t K, uint32_t box_rows,
+                       uint32_t kpb) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn || K % 128 != 0) return false;
+  const cuuint64_t dims[3] = {128, rows, K / 128};
+  const cuuint64_t strides[2] = {K, 128};
+  const cuuint32_t box[3] = {128, box_rows, kpb};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // ------------------------------------------------------------ workspace layout
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 struct Layout {
   int path = 0;
-  int Kw = 0, R = 0, rows_per_chunk = 0, ldo = 0, num_tiles = 0;
-  size_t part = 0, flags = 0, idx = 0, n_out = 0, counters = 0, sx = 0, xq = 0, xo = 0, wo = 0,
-         partials = 0, total = 0;
+  int Kw = 0, R = 0, rows_per_chunk = 0, ldo = 0;
+  size_t part = 0, flags = 0, idx = 0, n_out = 0, sx = 0, xq = 0, xo = 0, wo = 0, total = 0;
 };
 
 bool make_layout(int64_t T, int64_t N, int64_t K, int path, Layout* L) {
@@ -161,9 +191,6 @@ bool make_layout(int64_t T, int64_t N, int64_t K, int path, Layout* L) {
     return at;
   };
   if (path == LLMINT8_PATH_GEMV) {
-    L->num_tiles = static_cast<int>((N + gemv::BM - 1) / gemv::BM);
-    L->counters = take(sizeof(int32_t) * (L->num_tiles ? L->num_tiles : 1));
-    L->partials = take(sizeof(int32_t) * gemv::MAX_CTAS * 2 * gemv::SLOT_INTS);
     L->idx = take(sizeof(int32_t) * K);
     L->n_out = take(sizeof(int32_t));
     L->sx = take(sizeof(float) * LLMINT8_GEMV_MAX_T);
@@ -239,19 +266,17 @@ struct Prep {
   int32_t* n_out;
 };
 
-// Activation stages.  Decode: one latency-oriented kernel (it also zeroes
-// the GEMV's tile counters when `ncounters` > 0).  Prefill: detect, compact,
+// Activation stages.  Decode: one latency-oriented kernel.  Prefill: detect, compact,
 // quantize + gathers (the W gather only when W != nullptr).
 int launch_prep(const Layout& L, const uint16_t* X, int T, int K, const uint16_t* W, int N, float tau,
-                uint8_t* ws, const Prep& out, cudaStream_t st, int ncounters = 0) {
+                uint8_t* ws, const Prep& out, cudaStream_t st) {
   uint32_t* flags = reinterpret_cast<uint32_t*>(ws + L.flags);
   cudaError_t e;
   if (L.path == LLMINT8_PATH_GEMV) {
-    int32_t* counters = reinterpret_cast<int32_t*>(ws + L.counters);
     auto k = T <= 1 ? decode_prep_kernel<1> : T <= 2 ? decode_prep_kernel<2> : T <= 4 ? decode_prep_kernel<4>
            : T <= 8 ? decode_prep_kernel<8> : decode_prep_kernel<16>;
     e = launch_ex(k, dim3(kDecodeCtas), dim3(kDecodeThreads), 0, st, true, kDecodeCtas, X, T, K, tau, out.xq,
-                  out.sx, out.idx, out.n_out, counters, ncounters);
+                  out.sx, out.idx, out.n_out);
     return e == cudaSuccess ? LLMINT8_OK : LLMINT8_ERR_CUDA;
   }
   uint32_t* part = reinterpret_cast<uint32_t*>(ws + L.part);
@@ -329,27 +354,35 @@ int matmul_impl(const void* Xv, int64_t T, int64_t K, const int8_t* Wq, const fl
     p.N = n;
     p.K = k;
     p.KB = (k + gemv::BK - 1) / gemv::BK;
-    p.num_tiles = L.num_tiles;
-    p.units = p.num_tiles * p.KB;
-    int grid = num_sms < gemv::MAX_CTAS ? num_sms : gemv::MAX_CTAS;
-    if (grid > p.units) grid = p.units;
-    p.grid = grid;
+    // Row slabs: every CTA takes CH chunks of H rows (a multiple of 8) over
+    // all of K, about N / SMs rows in all, so the grid fills the SMs with
+    // equal shares.  With K % 128 == 0 one copy brings KPB k-blocks of each
+    // row (3-D tensor maps); otherwise one k-block (2-D maps, which zero the
+    // ragged tail of K).
+    const int per = (n + num_sms - 1) / num_sms;
+    p.CH = (per + gemv::BM - 1) / gemv::BM;
+    p.H = ((per + p.CH - 1) / p.CH + 7) / 8 * 8;
+    const int grid = (n + p.CH * p.H - 1) / (p.CH * p.H);
+    p.kpb3d = (k % gemv::BK) == 0 ? 1 : 0;
+    p.KPB = p.kpb3d ? gemv::kpb_for_rows(p.H) : 1;
+    p.NU = (p.KB + p.KPB - 1) / p.KPB;
     p.sx = out.sx;
     p.sw = Wscale;
     p.X = X;
     p.W = W;
     p.idx = out.idx;
     p.n_out = out.n_out;
-    p.counters = reinterpret_cast<int32_t*>(ws + L.counters);
-    p.partials = reinterpret_cast<int32_t*>(ws + L.partials);
     p.Y = Y;
     p.acc_out = acc_out;
     p.wait_ns = wait_ns;
     CUtensorMap tw, tx;
-    if (!encode_2d(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT8, Wq, K, N, K, gemv::BK, gemv::BM) ||
-        !encode_2d(&tx, CU_TENSOR_MAP_DATA_TYPE_UINT8, out.xq, K, T, K, gemv::BK, gemv::NT))
-      return LLMINT8_ERR_CUDA;
-    rc = launch_prep(L, X, t, k, W, n, threshold, ws, out, st, p.num_tiles);
+    const bool maps_ok =
+        p.kpb3d ? encode_kblocks_3d(&tw, Wq, N, K, static_cast<uint32_t>(p.H), static_cast<uint32_t>(p.KPB)) &&
+                      encode_kblocks_3d(&tx, out.xq, T, K, gemv::NT, static_cast<uint32_t>(p.KPB))
+                : encode_2d(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT8, Wq, K, N, K, gemv::BK, static_cast<uint32_t>(p.H)) &&
+                      encode_2d(&tx, CU_TENSOR_MAP_DATA_TYPE_UINT8, out.xq, K, T, K, gemv::BK, gemv::NT);
+    if (!maps_ok) return LLMINT8_ERR_CUDA;
+    rc = launch_prep(L, X, t, k, W, n, threshold, ws, out, st);
     if (rc != LLMINT8_OK) return rc;
     if (ev_begin && cudaEventRecord(ev_begin, st) != cudaSuccess) return LLMINT8_ERR_CUDA;
     void (*kern)(const CUtensorMap, const CUtensorMap, const gemv::Params) =
@@ -377,7 +410,23 @@ int matmul_impl(const void* Xv, int64_t T, int64_t K, const int8_t* Wq, const fl
   p.Y = Y;
   p.acc_out = acc_out;
   p.wait_ns = wait_ns;
-  const int num_n = (n + gemm::BN - 1) / gemm::BN;
+  // CTA pairs: the tile width whose tiles spread most evenly over the resident
+  // pairs, counting each tile's fixed cost as 32 more columns of work (a tie
+  // keeps the wider tile).
+  p.bn = gemm::BN;
+  if (pair) {
+    int64_t best = -1;
+    for (int bn : {256, 192, 128}) {
+      const int64_t tiles = static_cast<int64_t>(p.num_m) * ((n + bn - 1) / bn);
+      const int64_t rounds = (tiles + max_pairs - 1) / max_pairs;
+      const int64_t cost = rounds * (bn + 32);
+      if (best < 0 || cost < best) {
+        best = cost;
+        p.bn = bn;
+      }
+    }
+  }
+  const int num_n = (n + p.bn - 1) / p.bn;
   p.num_tiles = p.num_m * num_n;
   p.num_pairs = pair ? (p.num_tiles < max_pairs ? p.num_tiles : max_pairs) : 0;
   p.y_tma = (pair && n % 8 == 0) ? 1 : 0;
@@ -388,17 +437,17 @@ int matmul_impl(const void* Xv, int64_t T, int64_t K, const int8_t* Wq, const fl
   const uint16_t* xo = reinterpret_cast<const uint16_t*>(ws + L.xo);
   const uint16_t* wo = reinterpret_cast<const uint16_t*>(ws + L.wo);
   if (!encode_2d(&txq, CU_TENSOR_MAP_DATA_TYPE_UINT8, out.xq, K, T, K, gemm::BK, gemm::BM) ||
-      !encode_2d(&twq, CU_TENSOR_MAP_DATA_TYPE_UINT8, Wq, K, N, K, gemm::BK, pair ? gemm::BN / 2 : gemm::BN) ||
+      !encode_2d(&twq, CU_TENSOR_MAP_DATA_TYPE_UINT8, Wq, K, N, K, gemm::BK, pair ? p.bn / 2 : gemm::BN) ||
       !encode_2d(&txo, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, xo, L.ldo, T, 2ull * L.ldo, 64, gemm::BM) ||
       !encode_2d(&two, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, wo, L.ldo, N, 2ull * L.ldo, 64,
-                 pair ? gemm::BN / 2 : gemm::BN))
+                 pair ? p.bn / 2 : gemm::BN))
     return LLMINT8_ERR_CUDA;
   rc = launch_prep(L, X, t, k, W, n, threshold, ws, out, st);
   if (rc != LLMINT8_OK) return rc;
   if (ev_begin && cudaEventRecord(ev_begin, st) != cudaSuccess) return LLMINT8_ERR_CUDA;
   for (int r = 0; r < repeat; ++r) {
     const cudaError_t e =
-        pair ? launch_ex(gemm::gemm_pair_kernel, dim3(2 * p.num_pairs), dim3(gemm::THREADS),
+        pair ? launch_ex(gemm::gemm_pair_kernel, dim3(2 * p.num_pairs), dim3(gemm::P_THREADS),
                          gemm::P_SMEM_BYTES, st, true, 2, txq, twq, txo, two, ty, p)
              : launch(gemm::gemm_kernel, dim3(p.num_m * num_n), dim3(gemm::THREADS), gemm::SMEM_BYTES, st, true,
                       txq, twq, txo, two, p);
@@ -411,11 +460,11 @@ int matmul_impl(const void* Xv, int64_t T, int64_t K, const int8_t* Wq, const fl
 // ------------------------------------------------------------ allocation-free decode
 // Scratch for llmint8_matmul_decode_noalloc: one array per device that loads
 // the library, held until the process exits.  Sized for the decode path's
-// workspace at T <= 16, K <= kNoAllocMaxK, N <= kNoAllocMaxN (about 4.4 MB
-// used of 5 MiB; the stream-K partial slots are most of it).
+// workspace at T <= 16, K <= kNoAllocMaxK, N <= kNoAllocMaxN (about 0.33 MB
+// used of 1 MiB: the activation codes, their scales and the outlier list).
 constexpr int64_t kNoAllocMaxK = 16384;
 constexpr int64_t kNoAllocMaxN = 65536;
-constexpr size_t kNoAllocScratchBytes = 5u << 20;
+constexpr size_t kNoAllocScratchBytes = 1u << 20;
 static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
 
 struct NoAllocScratch {
@@ -569,8 +618,7 @@ int llmint8_matmul_decode_noalloc(const void* X, int64_t T, int64_t K, const int
   void* scratch = nullptr;
   rc = noalloc_scratch(&scratch);
   if (rc != LLMINT8_OK) return rc;
-  // The decode prep kernel zeroes the per-tile counters at the start of every
-  // call; every other scratch word is written before it is read.
+  // Every scratch word is written before it is read.
   return matmul_impl(X, T, K, Wq, Wscale, W, N, threshold, Y, scratch, kNoAllocScratchBytes,
                      LLMINT8_PATH_GEMV, Inspect{}, stream);
 }

@@ -313,8 +313,7 @@ constexpr int kDecodeMaxSlice = 65536 / 8 / kDecodeCtas;  // chunks per CTA at K
 template <int TMAX>
 __global__ void __launch_bounds__(kDecodeThreads, 4) decode_prep_kernel(
     const uint16_t* __restrict__ X, int T, int K, float tau, int8_t* __restrict__ Xq,
-    float* __restrict__ sx, int32_t* __restrict__ idx, int32_t* __restrict__ n_out,
-    int32_t* __restrict__ counters, int ncounters) {
+    float* __restrict__ sx, int32_t* __restrict__ idx, int32_t* __restrict__ n_out) {
   __shared__ uint8_t fm[kDecodeMaxSlice];
   __shared__ float red[kDecodeThreads / 32][TMAX];
   __shared__ float part[kDecodeCtas][TMAX];  // read in rank 0: every CTA's row maxima
@@ -334,8 +333,6 @@ __global__ void __launch_bounds__(kDecodeThreads, 4) decode_prep_kernel(
   const int items = myn * TMAX;
   const int t = tid % TMAX;
   const uint4* xrow = reinterpret_cast<const uint4*>(X + static_cast<int64_t>(t) * K) + c_begin;
-  for (int i = static_cast<int>(rank) * kDecodeThreads + tid; i < ncounters; i += kDecodeCtas * kDecodeThreads)
-    counters[i] = 0;
 
   // pass 1 (rounds are uniform across the CTA: the shuffles need whole warps)
   const int rounds = (items + kDecodeThreads * kDecodeInFlight - 1) / (kDecodeThreads * kDecodeInFlight);

@@ -378,7 +378,7 @@ def test_cuda_graph_replay_matches_direct_calls(L, oracle, path):
 @pytest.mark.parametrize("path", [1, 2])
 def test_profile_repeats_recompute_same_y(L, oracle, path):
     """The profiling entry relaunches the main kernel on one workspace; every
-    launch must recompute the same Y (the GEMV's tile counters reset themselves)."""
+    launch must recompute the same Y."""
     T = 7 if path == 1 else 150
     X, W = synth.random_case(T, 2048, 700, seed=60 + path, n_dims=4)
     Wd = dev(W)
