@@ -328,7 +328,7 @@ def time_main_kernel(wl: Workload, steps: int, flush) -> tuple[float, float]:
 
 
 def main_kernel_name(wl: Workload) -> str:
-    return "decode_call" if wl.unit == "GB/s" else "gemm_kernel"
+    return "decode_call" if wl.unit == "GB/s" else "gemm_pair_kernel"
 
 
 def roofline(wl: Workload, kern_ms: float, algo_per_launch: float, peaks: dict, traffic=None) -> dict:
@@ -345,7 +345,7 @@ def roofline(wl: Workload, kern_ms: float, algo_per_launch: float, peaks: dict, 
     peak = peaks["bf16_tflops"] * INT8_PER_BF16
     return {"bound": "tensor", "achieved": round(achieved, 1), "peak": round(peak, 1), "unit": "TOPS",
             "frac": round(achieved / peak, 4), "traffic": traffic,
-            "kernel": "gemm_kernel (tcgen05 kind::i8 + kind::f16)",
+            "kernel": "gemm_pair_kernel (persistent CTA pairs, tcgen05 cta_group::2 kind::i8 + kind::f16)",
             "peak_source": f"{peaks['source']} bf16_tflops (burst) x 2 (nominal int8/bf16 ratio)",
             "algo_ops_per_launch": int(algo_per_launch), "ms_per_launch": round(kern_ms, 5)}
 

@@ -29,11 +29,10 @@
 // Warp roles (192 threads): warp 0 lane 0 issues TMA; warp 1 lane 0 issues
 // tcgen05.mma and owns TMEM; warps 2-5 (128 threads = 128 TMEM lanes) compute
 // a chunk's outlier products while its weights stream, then drain its
-// accumulator.  Only PRE weight stages are requested before the prep kernel is
-// done: the SM's TMA unit serves copies in order, and the activation codes of
-// the first stages must not queue behind a long run of weight copies.  Two
-// 16-column accumulators let the MMA of one chunk overlap the epilogue of the
-// previous one.  Every wait is bounded.
+// accumulator.  The weight copies of the first PRE stages are issued before
+// the prep kernel is done (they do not depend on it), the activation codes of
+// those stages as soon as it is.  Two 16-column accumulators let the MMA of one
+// chunk overlap the epilogue of the previous one.  Every wait is bounded.
 #pragma once
 #include <cuda_fp16.h>
 #include "sm100.cuh"
@@ -46,7 +45,7 @@ constexpr int BK = 128;                    // K bytes per k-block (one 128 B swi
 constexpr int NT = 16;                     // tokens per MMA (MMA N)
 constexpr int KPB_MAX = 4;                 // k-blocks per stage
 constexpr int STAGES = 4;
-constexpr int PRE = 2;                     // weight stages requested before the prep kernel is done
+constexpr int PRE = STAGES;                // weight stages requested before the prep kernel is done
 constexpr int A_BYTES = 40 * 1024;         // Wq: KPB tiles of H x 128 bytes (H * 128 * KPB <= 40 KiB)
 constexpr int B_TILE = NT * BK;            // 2 KiB of activation codes per k-block
 constexpr int B_BYTES = KPB_MAX * B_TILE;
