@@ -322,8 +322,6 @@ __global__ void __launch_bounds__(kDecodeThreads, 4) decode_prep_kernel(
   __shared__ int s_off;
   __shared__ int scratch[33];
   pdl_launch_dependents();
-  cluster_sync();  // every CTA of the cluster has started before any remote access
-  pdl_wait();
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const uint32_t rank = cluster_ctarank();
   const int nchunk = K >> 3;
@@ -333,6 +331,14 @@ __global__ void __launch_bounds__(kDecodeThreads, 4) decode_prep_kernel(
   const int items = myn * TMAX;
   const int t = tid % TMAX;
   const uint4* xrow = reinterpret_cast<const uint4*>(X + static_cast<int64_t>(t) * K) + c_begin;
+  // Ask L2 for this thread's lines of X before waiting for the previous
+  // kernel: the loads after the wait then do not queue behind the GEMV's
+  // weight stream at DRAM.  A prefetch only reads (L2 stays coherent with
+  // any later write of X), so it is safe however X is produced.
+  for (int e = tid; e < items; e += kDecodeThreads)
+    if (t < T && (e / TMAX) % 8 == 0) prefetch_l2(xrow + e / TMAX);
+  cluster_sync();  // every CTA of the cluster has started before any remote access
+  pdl_wait();
 
   // pass 1 (rounds are uniform across the CTA: the shuffles need whole warps)
   const int rounds = (items + kDecodeThreads * kDecodeInFlight - 1) / (kDecodeThreads * kDecodeInFlight);
