@@ -183,6 +183,15 @@ def test_matmul_small(L, oracle, path, T, N, K, tau):
     run_full(L, oracle, X, W, tau, path)
 
 
+@pytest.mark.parametrize("T,N,K", [(3, 20011, 512), (16, 38000, 256), (1, 19000, 16)])
+def test_decode_many_rows_per_cta(L, oracle, T, N, K):
+    """N large enough that each GEMV CTA takes two or three chunks of rows
+    (N / 148 > 128), with a ragged last slab; K both a multiple of 128 (3-D
+    copies of several k-blocks) and not (2-D copies)."""
+    X, W = synth.random_case(T, K, N, seed=T + N, n_dims=3, mag=(6.0, 40.0))
+    run_full(L, oracle, X, W, 6.0, 1)
+
+
 @pytest.mark.parametrize("path", [1, 2])
 def test_tiny_config(L, oracle, path):
     w = synth.workload("tiny")
