@@ -226,7 +226,7 @@ class Workload:
         torch.cuda.synchronize()
         self.bytes_per_step = sum(c["bytes"] for c in self.calls)
         self.ops_per_step = sum(c["ops"] for c in self.calls)
-        self.launches_per_step = sum(2 if c["T"] <= 16 else 4 for c in self.calls)
+        self.launches_per_step = sum(L.llmint8_kernel_launches(c["T"], self.N, self.K) for c in self.calls)
         self.graph = None
 
     def capture(self):

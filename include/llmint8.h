@@ -91,6 +91,13 @@ LLMINT8_API size_t llmint8_workspace_bytes(int64_t T, int64_t N, int64_t K);
 /* Same for an explicit path (LLMINT8_PATH_*); 0 if the path cannot take T. */
 LLMINT8_API size_t llmint8_workspace_bytes_path(int64_t T, int64_t N, int64_t K, int path);
 
+/* How many kernels one llmint8_matmul call of this shape launches on `path`
+ * (no counterpart in the pages; for launch accounting): 2 for the decode path
+ * (prep + GEMV), 4 for the prefill path (detect, compact, quantize + gathers,
+ * GEMM).  0 for shapes the path rejects or T == 0 / N == 0.  Host-only:
+ * touches no device. */
+LLMINT8_API int llmint8_kernel_launches(int64_t T, int64_t N, int64_t K, int path);
+
 /*
  * Y = X * W^T by the LLM.int8() decomposition ('LLM quantization, part 2' §2.1;
  * '三、模型量化' Q4):

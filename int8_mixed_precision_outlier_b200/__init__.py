@@ -5,8 +5,8 @@ functions here are its Python binding.
 """
 from .llmint8 import (  # noqa: F401
     GEMV_MAX_T, PATH_AUTO, PATH_GEMM, PATH_GEMV, Int8Linear, LLMInt8Error, alloc_workspace,
-    header_functions, llmint8_detect_quantize, llmint8_matmul, llmint8_matmul_debug, llmint8_matmul_decode_noalloc, llmint8_matmul_intermediates,
-    llmint8_matmul_profile,
+    header_functions, llmint8_detect_quantize, llmint8_kernel_launches, llmint8_matmul, llmint8_matmul_debug,
+    llmint8_matmul_decode_noalloc, llmint8_matmul_intermediates, llmint8_matmul_profile,
     llmint8_quantize_weight, llmint8_selftest_timeout, llmint8_set_wait_limit_ns,
     llmint8_status_string, llmint8_sync_status, llmint8_version, llmint8_workspace_bytes,
     load_library,

@@ -534,6 +534,12 @@ size_t llmint8_workspace_bytes_path(int64_t T, int64_t N, int64_t K, int path) {
   return L.total;
 }
 
+int llmint8_kernel_launches(int64_t T, int64_t N, int64_t K, int path) {
+  Layout L;
+  if (T <= 0 || N <= 0 || !make_layout(T, N, K, path, &L)) return 0;
+  return L.path == LLMINT8_PATH_GEMV ? 2 : 4;
+}
+
 size_t llmint8_workspace_bytes(int64_t T, int64_t N, int64_t K) {
   return llmint8_workspace_bytes_path(T, N, K, LLMINT8_PATH_AUTO);
 }

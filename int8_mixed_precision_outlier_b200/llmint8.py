@@ -43,6 +43,7 @@ def _declare(lib):
         "llmint8_quantize_weight": (I, [P, I64, I64, P, P, P]),
         "llmint8_workspace_bytes": (SZ, [I64, I64, I64]),
         "llmint8_workspace_bytes_path": (SZ, [I64, I64, I64, I]),
+        "llmint8_kernel_launches": (I, [I64, I64, I64, I]),
         "llmint8_matmul": (I, [P, I64, I64, P, P, P, I64, F, P, P, SZ, P]),
         "llmint8_matmul_debug": (I, [P, I64, I64, P, P, P, I64, F, P, P, SZ, I, P, P, P, P, P, P]),
         "llmint8_matmul_profile": (I, [P, I64, I64, P, P, P, I64, F, P, P, SZ, I, I, P, P, P]),
@@ -117,6 +118,11 @@ def llmint8_workspace_bytes(T: int, N: int, K: int, path: int = PATH_AUTO) -> in
     if path == PATH_AUTO:
         return int(lib.llmint8_workspace_bytes(T, N, K))
     return int(lib.llmint8_workspace_bytes_path(T, N, K, path))
+
+
+def llmint8_kernel_launches(T: int, N: int, K: int, path: int = PATH_AUTO) -> int:
+    """Kernels one llmint8_matmul call of this shape launches (0 if rejected)."""
+    return int(load_library().llmint8_kernel_launches(T, N, K, path))
 
 
 def llmint8_set_wait_limit_ns(ns: int):

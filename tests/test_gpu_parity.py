@@ -183,6 +183,17 @@ def test_matmul_small(L, oracle, path, T, N, K, tau):
     run_full(L, oracle, X, W, tau, path)
 
 
+@pytest.mark.parametrize("T,N,K", [(1, 1000, 128), (2, 300, 4096), (3, 11008, 2048), (4, 513, 4096)])
+@pytest.mark.parametrize("tau", [6.0, 0.0, float("inf"), 30.0])
+def test_decode_small_t_thresholds(L, oracle, T, N, K, tau):
+    """Decode with T <= 4 and K % 128 == 0 (3-D weight copies): every
+    intermediate (Xq, sx, the outlier list, int32 acc) bit-exact, Y within
+    tolerance; tau = 0 makes every column an outlier (|O| = K), tau = inf none."""
+    assert L.llmint8_kernel_launches(T, N, K) == 2
+    X, W = synth.random_case(T, K, N, seed=T * 7 + K, n_dims=min(4, K), mag=(6.0, 50.0))
+    run_full(L, oracle, X, W, tau, 1)
+
+
 @pytest.mark.parametrize("T,N,K", [(3, 20011, 512), (16, 38000, 256), (1, 19000, 16)])
 def test_decode_many_rows_per_cta(L, oracle, T, N, K):
     """N large enough that each GEMV CTA takes two or three chunks of rows
