@@ -297,9 +297,11 @@ __global__ void __launch_bounds__(kQuantThreads) quant_gather_kernel(
 // OR across them, and each thread keeps one row's running absmax.
 //   pass 1: masks -> shared mask bytes; per-row absmax over regular columns
 //   exchange: each CTA writes its per-row maxima and its outlier count into
-//     rank 0's shared memory (distributed shared memory); after a cluster
-//     barrier every CTA forms sx[t] = max / 127 and its offset in the list
-//   pass 2: codes (X re-read from L2) -> Xq; this CTA's outlier indices
+//     every CTA's shared memory (distributed shared memory); after one
+//     cluster barrier every CTA forms sx[t] = max / 127 and its offset in the
+//     list from its own copies
+//   then: this CTA's outlier indices; codes (values kept in registers, or X
+//     re-read from L2) -> Xq
 // 256 threads and at most 64 registers per CTA let a CTA share an SM with a
 // GEMV CTA, so the cluster launches while the previous call's GEMV runs.  It
 // waits for its predecessor before touching memory and lets the GEMV launch at
@@ -316,8 +318,8 @@ __global__ void __launch_bounds__(kDecodeThreads, 4) decode_prep_kernel(
     float* __restrict__ sx, int32_t* __restrict__ idx, int32_t* __restrict__ n_out) {
   __shared__ uint8_t fm[kDecodeMaxSlice];
   __shared__ float red[kDecodeThreads / 32][TMAX];
-  __shared__ float part[kDecodeCtas][TMAX];  // read in rank 0: every CTA's row maxima
-  __shared__ int cnt[kDecodeCtas];           // read in rank 0: every CTA's outlier count
+  __shared__ float part[kDecodeCtas][TMAX];  // every CTA's row maxima (each CTA holds a copy)
+  __shared__ int cnt[kDecodeCtas];           // every CTA's outlier count (each CTA holds a copy)
   __shared__ float s_sx[TMAX], s_inv[TMAX];
   __shared__ int s_off;
   __shared__ int scratch[33];
@@ -366,24 +368,34 @@ __global__ void __launch_bounds__(kDecodeThreads, 4) decode_prep_kernel(
 #pragma unroll
   for (int o = 16; o >= TMAX; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
   if (lane < TMAX) red[warp][lane] = m;
-  __syncthreads();
+  __syncthreads();  // red and fm complete
+  // This CTA's outlier positions, ascending: thread i owns chunks
+  // [i*cpt, (i+1)*cpt); the scan gives its place among this CTA's outliers.
+  const int cpt = (myn + kDecodeThreads - 1) / kDecodeThreads;
+  const int c0 = tid * cpt;
   int count = 0;
-  for (int i = tid; i < myn; i += kDecodeThreads) count += __popc(static_cast<uint32_t>(fm[i]));
+  for (int i = 0; i < cpt; ++i)
+    if (c0 + i < myn) count += __popc(static_cast<uint32_t>(fm[c0 + i]));
   int my_total;
-  block_exclusive_scan(count, scratch, &my_total);
-  if (tid < TMAX) {
+  const int pos_local = block_exclusive_scan(count, scratch, &my_total);
+  // Every CTA sends its row maxima and outlier count to every CTA of the
+  // cluster, so that after one cluster barrier each reads its own copies
+  // (and no CTA's shared memory is read after it may have exited).
+  if (tid < TMAX * kDecodeCtas) {
+    const int tt = tid % TMAX, dst = tid / TMAX;
     float pm = 0.0f;
 #pragma unroll
-    for (int w = 0; w < kDecodeThreads / 32; ++w) pm = fmaxf(pm, red[w][tid]);
-    st_cluster_f32(map_shared_rank(&part[rank][tid], 0), pm);
+    for (int w = 0; w < kDecodeThreads / 32; ++w) pm = fmaxf(pm, red[w][tt]);
+    st_cluster_f32(map_shared_rank(&part[rank][tt], static_cast<uint32_t>(dst)), pm);
   }
-  if (tid == 0) st_cluster_u32(map_shared_rank(&cnt[rank], 0), static_cast<uint32_t>(my_total));
+  if (tid >= 224 && tid < 224 + kDecodeCtas)
+    st_cluster_u32(map_shared_rank(&cnt[rank], static_cast<uint32_t>(tid - 224)), static_cast<uint32_t>(my_total));
   cluster_sync();
 
   if (tid < TMAX) {
     float mm = 0.0f;
 #pragma unroll
-    for (int r = 0; r < kDecodeCtas; ++r) mm = fmaxf(mm, ld_cluster_f32(map_shared_rank(&part[r][tid], 0)));
+    for (int r = 0; r < kDecodeCtas; ++r) mm = fmaxf(mm, part[r][tid]);
     const float s = __fdiv_rn(mm, 127.0f);
     s_sx[tid] = s;
     s_inv[tid] = scale_reciprocal(s);
@@ -392,16 +404,24 @@ __global__ void __launch_bounds__(kDecodeThreads, 4) decode_prep_kernel(
   if (tid == 32) {
     int off = 0, total = 0;
     for (int r = 0; r < kDecodeCtas; ++r) {
-      const int c = static_cast<int>(ld_cluster_u32(map_shared_rank(&cnt[r], 0)));
+      const int c = cnt[r];
       off += r < static_cast<int>(rank) ? c : 0;
       total += c;
     }
     s_off = off;
     if (rank == 0) *n_out = total;
   }
-  cluster_sync();  // rank 0's shared memory stays valid until every CTA has read it
+  __syncthreads();  // s_sx, s_inv, s_off
 
-  // pass 2
+  // outlier indices
+  int pos = s_off + pos_local;
+  for (int i = 0; i < cpt; ++i) {
+    const int c = c0 + i;
+    if (c >= myn) break;
+    for (uint32_t f = fm[c]; f; f &= f - 1) idx[pos++] = (c_begin + c) * 8 + (__ffs(f) - 1);
+  }
+
+  // pass 2: codes
   const float st = s_sx[t], it = s_inv[t];
   for (int r = 0; r < rounds; ++r) {
     const int base = r * kDecodeThreads * kDecodeInFlight + tid;
@@ -419,25 +439,6 @@ __global__ void __launch_bounds__(kDecodeThreads, 4) decode_prep_kernel(
         const int c = e / TMAX;
         reinterpret_cast<uint2*>(Xq + static_cast<int64_t>(t) * K)[c_begin + c] = quant8(v[u], st, it, fm[c]);
       }
-    }
-  }
-
-  // this CTA's outlier indices, ascending: thread i owns chunks [i*cpt, (i+1)*cpt)
-  const int cpt = (myn + kDecodeThreads - 1) / kDecodeThreads;
-  const int c0 = tid * cpt;
-  count = 0;
-  for (int i = 0; i < cpt; ++i)
-    if (c0 + i < myn) count += __popc(static_cast<uint32_t>(fm[c0 + i]));
-  int unused;
-  int pos = s_off + block_exclusive_scan(count, scratch, &unused);
-  for (int i = 0; i < cpt; ++i) {
-    const int c = c0 + i;
-    if (c >= myn) break;
-    uint32_t f = fm[c];
-    while (f) {
-      const int b = __ffs(f) - 1;
-      idx[pos++] = (c_begin + c) * 8 + b;
-      f &= f - 1;
     }
   }
 }
