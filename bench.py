@@ -79,16 +79,45 @@ def load_peaks() -> dict:
         return dict(FALLBACK, source="fallback")
 
 
+def _strip_comments(src: str) -> str:
+    """C/C++ source with // and /* */ comments removed and each remaining line
+    stripped of surrounding whitespace; string and character literals are
+    kept as they are."""
+    out = []
+    i, n = 0, len(src)
+    while i < n:
+        c = src[i]
+        if c in "\"'":
+            j = i + 1
+            while j < n and src[j] != c:
+                j += 2 if src[j] == "\\" else 1
+            out.append(src[i:j + 1])
+            i = j + 1
+        elif src.startswith("//", i):
+            j = src.find("\n", i)
+            i = n if j < 0 else j
+        elif src.startswith("/*", i):
+            j = src.find("*/", i + 2)
+            i = n if j < 0 else j + 2
+        else:
+            out.append(c)
+            i += 1
+    lines = (ln.strip() for ln in "".join(out).splitlines())
+    return "\n".join(ln for ln in lines if ln)
+
+
 def source_digest() -> str:
-    """sha256 over the CUDA sources: a recorded ncu traffic figure is only used
-    while the kernels it was measured on are unchanged."""
+    """sha256 over the code of the CUDA sources (comments and blank lines
+    excluded): a recorded ncu traffic figure is only used while the kernels it
+    was measured on are unchanged."""
     import glob
     import hashlib
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "int8_mixed_precision_outlier_b200", "csrc")
     for f in sorted(glob.glob(os.path.join(csrc, "*.cu*"))):
-        with open(f, "rb") as fh:
-            h.update(os.path.basename(f).encode() + b"\0" + fh.read())
+        with open(f, encoding="utf-8") as fh:
+            code = _strip_comments(fh.read())
+        h.update(os.path.basename(f).encode() + b"\0" + code.encode())
     return h.hexdigest()[:16]
 
 

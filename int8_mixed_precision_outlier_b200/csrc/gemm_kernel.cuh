@@ -1,7 +1,9 @@
 // gemm_kernel.cuh -- prefill-shaped LLM.int8() matmul on the 5th-generation
-// tensor cores.
+// tensor cores: gemm_pair_kernel (further below) for T > 128, persistent 2-CTA
+// clusters with tcgen05 cta_group::2; gemm_kernel for 17 <= T <= 128.
 //
-// One CTA computes a BM x BN tile of Y = X * W^T:
+// Both compute tiles of Y = X * W^T; in gemm_kernel one CTA takes a BM x BN
+// tile:
 //   acc = Xq[m-tile, :] * Wq[n-tile, :]^T     tcgen05.mma kind::i8 -> int32 TMEM
 //   yo  = Xo[m-tile, :] * Wo[n-tile, :]^T     tcgen05.mma kind::f16 -> fp32 TMEM
 //   Y   = fp16( acc * sx[t] * sw[n] + yo )    epilogue (tcgen05.ld -> registers)
