@@ -329,9 +329,9 @@ def time_main_kernel(wl: Workload, steps: int, flush) -> tuple[float, float]:
     """Average duration of the roofline unit on cold L2, as in the timed steps
     (flush before each step, the step's calls in order, one launch each).
 
-    Decode: one whole call, decode_prep_kernel then gemv_kernel.  The prep
-    kernel starts the weight stream into L2 for the GEMV, so the two share the
-    HBM time and are timed together.  Prefill: the GEMM launch alone (events
+    Decode: one whole call, decode_prep_kernel then gemv_kernel.  The GEMV
+    launches while the prep kernel runs and starts its weight stream then, so
+    the two share the HBM time and are timed together.  Prefill: the GEMM launch alone (events
     between the activation kernels and it).  Returns (ms per unit, algorithmic
     bytes or ops per unit)."""
     import torch
@@ -366,8 +366,8 @@ def roofline(wl: Workload, kern_ms: float, algo_per_launch: float, peaks: dict, 
         peak = peaks["hbm_gbs"]
         return {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                 "frac": round(achieved / peak, 4), "traffic": traffic,
-                "kernel": "decode_prep_kernel + gemv_kernel (one call; the GEMV streams the weights, "
-                          "the prep kernel starts that stream into L2)",
+                "kernel": "decode_prep_kernel + gemv_kernel (one call; the GEMV streams the weights "
+                          "and starts that stream while the prep kernel runs)",
                 "peak_source": f"{peaks['source']} hbm_gbs (copy, burst)",
                 "algo_bytes_per_launch": int(algo_per_launch), "ms_per_launch": round(kern_ms, 5)}
     achieved = algo_per_launch / (kern_ms * 1e-3) / 1e12

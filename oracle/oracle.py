@@ -41,16 +41,22 @@ _LIBPATH = os.path.join(_HERE, "liboracle.so")
 _LOCK = threading.Lock()
 _LIB = None
 
-_CFLAGS = ["-O2", "-std=c11", "-fno-fast-math", "-ffp-contract=off", "-fopenmp", "-fPIC",
+CFLAGS = ["-O2", "-std=c11", "-fno-fast-math", "-ffp-contract=off", "-fopenmp", "-fPIC",
            "-shared", "-Wall", "-Wextra"]
 
 
 def build(force: bool = False) -> str:
-    """Compile liboracle.so next to its source (gcc, OpenMP)."""
+    """Compile liboracle.so next to its source (gcc, OpenMP).  With
+    LLMINT8_ORACLE_LIB set, that library is used as it is instead: the
+    mutation tests compile copies of the source with planted mistakes and run
+    the pins against them."""
+    override = os.environ.get("LLMINT8_ORACLE_LIB")
+    if override:
+        return override
     if force or not os.path.exists(_LIBPATH) or os.path.getmtime(_LIBPATH) < max(
             os.path.getmtime(_SRC), os.path.getmtime(os.path.join(_HERE, "llmint8_oracle.h"))):
         tmp = _LIBPATH + f".tmp{os.getpid()}"
-        subprocess.check_call(["gcc", *_CFLAGS, "-o", tmp, _SRC, "-lm"])
+        subprocess.check_call(["gcc", *CFLAGS, "-o", tmp, _SRC, "-lm"])
         os.replace(tmp, _LIBPATH)
     return _LIBPATH
 
