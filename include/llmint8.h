@@ -113,6 +113,10 @@ LLMINT8_API int llmint8_kernel_launches(int64_t T, int64_t N, int64_t K, int pat
  * workspace: device scratch of at least llmint8_workspace_bytes(T, N, K) bytes,
  * owned by the caller, contents on entry ignored; calls that share a workspace
  * must be ordered on one stream.  The outlier set never returns to the host.
+ * The kernels launch with programmatic dependent launch and start reading Wq
+ * before the kernel queued ahead of them on `stream` is done (X, W, Wscale
+ * and the workspace only after it): Wq must not be written by a kernel that
+ * lets its dependents launch before its own writes are complete.
  * T >= 1, N >= 1, K >= 16, K % 16 == 0, K * 127 * 127 < 2^31.
  */
 LLMINT8_API int llmint8_matmul(const void* X, int64_t T, int64_t K, const int8_t* Wq, const float* Wscale,
