@@ -3,13 +3,14 @@
 Integer stages (Wq, Wscale, outlier set, Xq, sx, int32 acc) must match bit for
 bit; Y must satisfy |Y_gpu - Y_oracle| <= 1e-3 max|Y_oracle| + 1 fp16 ulp.
 Small cases compare every element; the full-size workloads compare every
-integer stage in full and Y / acc on sampled rows, computed by the oracle one
-row at a time.
+integer stage in full (the int32 accumulator of every row by Freivalds'
+projection check against the oracle's codes) and Y / acc element by element
+on sampled rows, computed by the oracle one row at a time.
 """
 import numpy as np
 import pytest
 
-from gpu_helpers import assert_equal, assert_y_close
+from gpu_helpers import assert_acc_exact, assert_equal, assert_y_close, projected_weights
 from int8_mixed_precision_outlier_b200 import synth
 
 pytestmark = pytest.mark.gpu
@@ -244,7 +245,9 @@ def sampled_rows(T, seed):
 
 
 def run_sampled(L, oracle, X, W, taus, seed=0):
-    """Full-size check: every integer stage in full, Y and acc on sampled rows."""
+    """Full-size check: every integer stage in full (acc of all rows by
+    random projections, exact in int64), Y and acc element by element on
+    sampled rows."""
     T, K = X.shape
     N = W.shape[0]
     Wq_o, sw_o = oracle.quantize_weight(W)
@@ -255,6 +258,7 @@ def run_sampled(L, oracle, X, W, taus, seed=0):
     ws = L.alloc_workspace(T, N, K, "cuda")
     acc = torch.empty((T, N), dtype=torch.int32, device="cuda")
     rows = sampled_rows(T, seed)
+    proj = projected_weights(Wq_o, seed=seed)
     for tau in taus:
         flag = oracle.detect_outliers(X, tau)
         idx_o = oracle.compact(flag)
@@ -270,7 +274,9 @@ def run_sampled(L, oracle, X, W, taus, seed=0):
         acc_o = oracle.int8_gemm(np.ascontiguousarray(Xq_o[rows]), Wq_o)
         yo_o = oracle.outlier_gemm(Xs, W, idx_o)
         Y_o = oracle.dequant_combine(acc_o, sx_o[rows], sw_o, yo_o)
-        assert_equal(host(acc[rows]), acc_o, f"acc rows tau={tau}")
+        acc_h = host(acc)
+        assert_acc_exact(acc_h, Xq_o, proj, f"acc all rows tau={tau}")
+        assert_equal(acc_h[rows], acc_o, f"acc rows tau={tau}")
         assert_y_close(host(Y[rows]), Y_o, f"Y rows tau={tau}")
         # a property at any size: Y is finite and the last row was written
         assert torch.isfinite(Y).all()
