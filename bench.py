@@ -466,6 +466,12 @@ def run_reference(args):
     rank, world, _ = dist_env()
     if rank != 0:
         return 0
+    if world > 1:
+        # rank 0 works alone: give the oracle every host core, not the one
+        # OpenMP thread per rank that the launcher sets by default (torch is
+        # loaded already and the oracle shares its OpenMP runtime)
+        import torch
+        torch.set_num_threads(len(os.sched_getaffinity(0)))
     calls, sample, unit = oracle_sample(args.workload)
     # One step to warm caches and threads and to size the sample: exactly
     # `steps` timed steps (after `warmup` untimed ones) fit in the budget.

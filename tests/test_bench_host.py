@@ -96,3 +96,18 @@ def test_reference_arm_prints_the_contract_line():
     assert cb["kind"] == "oracle" and cb["value"] == line["value"] and cb["cores"] >= 1 and cb["sample"]
     assert line["e2e"] == {"value": line["value"], "unit": "GB/s", "h2d_bytes_per_step": 0,
                            "d2h_bytes_per_step": 0}
+
+
+def test_reference_arm_under_torchrun_prints_once_with_all_cores():
+    """Two ranks: rank 0 alone times the oracle, on every host core; rank 1
+    exits 0 without work."""
+    r = subprocess.run([sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node", "2",
+                        "--master-addr", "127.0.0.1", "--master-port", "29541", "bench.py", "--impl",
+                        "reference", "--gpus", "2", "--steps", "3", "--warmup", "3", "--ref-budget-s", "2"],
+                       cwd=ROOT, capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stderr[-3000:]
+    lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1
+    line = json.loads(lines[0])
+    assert line["n_gpus"] == 2 and line["steps"] == 3
+    assert line["cpu_baseline"]["cores"] == len(os.sched_getaffinity(0))
