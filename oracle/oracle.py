@@ -15,7 +15,7 @@ Method (pages on LLM quantization, sections theirs):
   * '量化压缩实战' (tqpw.cn) §2.1: scale = max_val/127, round, clip; worked
     example [0.0023,-1.5,4.7,0.001,8.9,-2.3] -> [0,-21,67,0,127,-33].
 
-Readings where the pages are silent or ambiguous (each is listed in the design doc):
+Readings where the pages are silent or ambiguous:
 outlier test |x| >= tau on any row of this call; per-row activation scale over
 the non-outlier columns; weight scale over all columns; round half to even in
 binary32 on fl(x/s); clamp to [-127, 127]; s = 0 gives code 0; the fp part and
