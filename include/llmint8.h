@@ -60,8 +60,10 @@ typedef enum {
 /* Kernel path of llmint8_matmul.  AUTO takes GEMV for T <= 16, else GEMM. */
 enum {
   LLMINT8_PATH_AUTO = 0,
-  LLMINT8_PATH_GEMV = 1, /* decode: weight-streaming split-K tcgen05 (T <= 16 only)     */
-  LLMINT8_PATH_GEMM = 2  /* prefill: TMA-fed tcgen05 int8 GEMM + fp16 outlier GEMM      */
+  LLMINT8_PATH_GEMV = 1, /* decode: one prep kernel + a weight-streaming tcgen05 GEMV,
+                            each CTA a slab of output rows over all of K (T <= 16 only) */
+  LLMINT8_PATH_GEMM = 2  /* prefill: activation kernels + a TMA-fed tcgen05 int8 GEMM
+                            with the fp16 outlier GEMM in a second TMEM accumulator      */
 };
 
 /* Largest T the decode path takes. */
@@ -170,7 +172,7 @@ LLMINT8_API int llmint8_detect_quantize(const void* X, int64_t T, int64_t K, flo
 
 /*
  * llmint8_matmul for decode shapes (T <= 16) without a caller workspace and
- * without allocating anything.  The paper has no counterpart: this entry
+ * without allocating anything.  The pages have no counterpart: this entry
  * serves callers that cannot call cudaMalloc, such as a host program that owns
  * all device memory through its own pool (a library may not take memory behind
  * its back) or a latency-critical loop where an allocation could stall the
