@@ -106,6 +106,18 @@ def test_validation_before_any_device_call(lib):
     assert lib.llmint8_selftest_timeout(10, None) == -1
 
 
+def test_noalloc_limits_checked_before_any_device_call(lib):
+    A = _fake(0x10000)
+    f = lib.llmint8_matmul_decode_noalloc
+    assert f(A, 17, 64, A, A, A, 8, 6.0, A, None) == -1        # T > 16: not a decode shape
+    assert f(A, 4, 16384 + 16, A, A, A, 8, 6.0, A, None) == -1  # K past the scratch limit
+    assert f(A, 4, 64, A, A, A, 65536 + 1, 6.0, A, None) == -1  # N past the limit
+    assert f(A, 4, 72, A, A, A, 8, 6.0, A, None) == -1          # K % 16 != 0
+    assert f(A, -1, 64, A, A, A, 8, 6.0, A, None) == -1
+    assert f(None, 0, 64, A, A, A, 8, 6.0, A, None) == 0        # empty problems are no-ops
+    assert f(A, 4, 64, A, A, A, 0, 6.0, A, None) == 0
+
+
 def test_missing_library_fails_loudly(tmp_path):
     from int8_mixed_precision_outlier_b200 import llmint8 as B
     with pytest.raises(OSError):
