@@ -379,8 +379,10 @@ def roofline(wl: Workload, kern_ms: float, algo_per_launch: float, peaks: dict, 
             "algo_ops_per_launch": int(algo_per_launch), "ms_per_launch": round(kern_ms, 5)}
 
 
-def e2e_steps(wl: Workload, steps: int, warmup: int, flush) -> dict:
-    """The public call with host buffers: pinned H2D of X, the matmul, D2H of Y."""
+def e2e_steps(wl: Workload, steps: int, warmup: int, flush, world: int = 1) -> dict:
+    """The public call with host buffers: pinned H2D of X, the matmul, D2H of Y.
+    Every rank runs it; the value is all ranks' units over the slowest rank's
+    time, and the copy bytes are the whole job's."""
     import torch
     L = wl.L
     hx = [torch.from_numpy(c["host_X"]).pin_memory() for c in wl.calls]
@@ -392,12 +394,15 @@ def e2e_steps(wl: Workload, steps: int, warmup: int, flush) -> dict:
             L.llmint8_matmul(c["X"], c["Wq"], c["sw"], c["W"], c["tau"], c["ws"], c["Y"])
             y.copy_(c["Y"], non_blocking=True)
 
-    total_ms, _ = time_steps(wl, steps, warmup, 1, flush, run=run)
-    h2d = sum(x.numel() * 2 for x in hx)
-    d2h = sum(y.numel() * 2 for y in hy)
-    return {"value": round(wl.metric_value(total_ms * 1e-3, steps), 2), "unit": wl.unit,
+    total_ms, _ = time_steps(wl, steps, warmup, world, flush, run=run)
+    t_max = reduce_max(total_ms, world)
+    units = reduce_sum((wl.bytes_per_step if wl.unit == "GB/s" else wl.ops_per_step) * steps, world)
+    value = units / (t_max * 1e-3) / (1e9 if wl.unit == "GB/s" else 1e12)
+    h2d = sum(x.numel() * 2 for x in hx) * world
+    d2h = sum(y.numel() * 2 for y in hy) * world
+    return {"value": round(value, 2), "unit": wl.unit,
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-            "ms_per_step": round(total_ms / steps, 5)}
+            "ms_per_step": round(t_max / steps, 5)}
 
 
 # ----------------------------------------------------------------- CPU oracle
@@ -549,8 +554,7 @@ def run_ours(args):
         "gpu_launches": wl.launches_per_step * args.steps,
         "clocks": clocks, "device_status": L.llmint8_status_string(status),
     }
-    if rank == 0 and world == 1:
-        line["e2e"] = e2e_steps(wl, args.steps, args.warmup, flush)
+    line["e2e"] = e2e_steps(wl, args.steps, args.warmup, flush, world)  # collective: every rank
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         calls, sample, unit = oracle_sample(args.workload)
         v, done, dt, cores = run_oracle(calls, unit, 1000, args.cpu_budget_s)
