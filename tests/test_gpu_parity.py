@@ -204,6 +204,17 @@ def test_decode_many_rows_per_cta(L, oracle, T, N, K):
     run_full(L, oracle, X, W, 6.0, 1)
 
 
+@pytest.mark.parametrize("path,T", [(1, 16), (1, 1), (2, 200)])
+def test_maximum_k(L, oracle, path, T):
+    """K = 65536, the largest K the library takes: the decode prep kernel's
+    per-CTA slice is full (1024 chunks of 8 columns), the GEMV streams 128
+    stages per row slab, the GEMM runs 512 k-blocks per tile."""
+    assert L.llmint8_workspace_bytes(T, 300, 65536) > 0
+    assert L.llmint8_workspace_bytes(T, 300, 65536 + 16) == 0
+    X, W = synth.random_case(T, 65536, 300, seed=T + 65536, n_dims=6, mag=(6.0, 50.0))
+    run_full(L, oracle, X, W, 6.0, path)
+
+
 @pytest.mark.parametrize("path", [1, 2])
 def test_tiny_config(L, oracle, path):
     w = synth.workload("tiny")
