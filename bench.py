@@ -38,6 +38,7 @@ from int8_mixed_precision_outlier_b200 import synth  # noqa: E402
 METRIC = "LLM.int8 matmul effective TOPS (2TNK/s) vs int8 TC peak; decode GEMV HBM GB/s"
 FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 INT8_PER_BF16 = 2.0  # nominal dense ratio: 4.5 POPS int8 / 2.25 PFLOPS bf16
+PUBLISHED = {"hbm_gbs": 8000.0, "int8_tops": 4500.0}  # B200 data-sheet figures (dense), for context
 THRESHOLD = 6.0
 FLUSH_BYTES = 256 << 20
 
@@ -369,6 +370,7 @@ def roofline(wl: Workload, kern_ms: float, algo_per_launch: float, peaks: dict, 
                 "kernel": "decode_prep_kernel + gemv_kernel (one call; the GEMV streams the weights "
                           "and starts that stream while the prep kernel runs)",
                 "peak_source": f"{peaks['source']} hbm_gbs (copy, burst)",
+                "frac_of_published": round(achieved / PUBLISHED["hbm_gbs"], 4),
                 "algo_bytes_per_launch": int(algo_per_launch), "ms_per_launch": round(kern_ms, 5)}
     achieved = algo_per_launch / (kern_ms * 1e-3) / 1e12
     peak = peaks["bf16_tflops"] * INT8_PER_BF16
@@ -376,6 +378,7 @@ def roofline(wl: Workload, kern_ms: float, algo_per_launch: float, peaks: dict, 
             "frac": round(achieved / peak, 4), "traffic": traffic,
             "kernel": "gemm_pair_kernel (persistent CTA pairs, tcgen05 cta_group::2 kind::i8 + kind::f16)",
             "peak_source": f"{peaks['source']} bf16_tflops (burst) x 2 (nominal int8/bf16 ratio)",
+            "frac_of_published": round(achieved / PUBLISHED["int8_tops"], 4),
             "algo_ops_per_launch": int(algo_per_launch), "ms_per_launch": round(kern_ms, 5)}
 
 
