@@ -7,7 +7,7 @@ the same recipes.
 
 The value distributions follow what the pages say about activations of 7B-70B
 models: about 99.9% of activations lie in [-1, 1], while a few fixed feature
-dimensions (about 0.1% of them, "a few dozen") carry values 20-100x larger on
+dimensions (about 0.1% of them, a few dozen at most) carry values 20-100x larger on
 almost every token ('LLM quantization, part 2' (hncyxsy.com) §1; '三、模型量化'
 (lowentro.cn) Q4 and Q11).  Weights are zero-mean normal.
 
