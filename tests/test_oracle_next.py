@@ -273,6 +273,29 @@ def test_reconstructed_weight_is_the_fp16_of_the_binary32_product(nx):
         assert got.view(np.uint16) == want.view(np.uint16), (q, s)
 
 
+def test_reconstruction_rounds_twice(nx):
+    """The product is rounded to binary32 first, then to fp16: where the exact
+    product sits just above an fp16 half-way point but its binary32 rounding
+    lands on it, ties-to-even takes the lower neighbour (one rounding of the
+    exact product would take the upper one)."""
+    found = 0
+    for q in (3, 5, 7, 9, 11, 13, 101, 127):
+        for h in range(0x3c01, 0x3c80, 2):                       # fp16 values in [1, 1.25), odd mantissa
+            lo = np.uint16(h - 1).view(np.float16)                 # even neighbour below
+            hi = np.uint16(h).view(np.float16)
+            m = (Fraction(float(lo)) + Fraction(float(hi))) / 2   # the half-way point
+            s = np.float32(float(m) / q)
+            for _ in range(4):
+                exact = Fraction(float(s)) * q
+                if exact > m and np.float32(float(s) * q) == np.float32(float(m)):
+                    got = nx.reconstruct_weight(q, s)
+                    assert got.view(np.uint16) == lo.view(np.uint16), (q, h)
+                    found += 1
+                    break
+                s = np.nextafter(s, np.float32(1))
+    assert found >= 5
+
+
 def test_full_store_equals_the_fp16_weight(nx, oracle):
     X, W = synth.random_case(10, 128, 37, seed=12, n_dims=5)
     Wq, sw = oracle.quantize_weight(W)
