@@ -180,15 +180,26 @@ void onext_fp8_quantize_activations(const uint16_t* X, int64_t T, int64_t K, con
 }
 
 void onext_fp8_gemm(const uint8_t* Xq, const uint8_t* Wq, int64_t T, int64_t N, int64_t K, double* acc) {
+  /* Each code is decoded once into a binary64 copy; the products and sums
+   * are the same (and exact, see next_oracle.h) in any order. */
+  double* xd = (double*)malloc(sizeof(double) * (size_t)(T * K > 0 ? T * K : 1));
+  double* wd = (double*)malloc(sizeof(double) * (size_t)(N * K > 0 ? N * K : 1));
+  if (!xd || !wd) {
+    for (int64_t i = 0; i < T * N; ++i) acc[i] = NAN;
+    free(xd); free(wd);
+    return;
+  }
+  for (int64_t i = 0; i < T * K; ++i) xd[i] = (double)onext_e4m3_to_float(Xq[i]);
+  for (int64_t i = 0; i < N * K; ++i) wd[i] = (double)onext_e4m3_to_float(Wq[i]);
 #pragma omp parallel for collapse(2) schedule(static)
   for (int64_t t = 0; t < T; ++t) {
     for (int64_t n = 0; n < N; ++n) {
       double s = 0.0;
-      for (int64_t k = 0; k < K; ++k)
-        s += (double)onext_e4m3_to_float(Xq[t * K + k]) * (double)onext_e4m3_to_float(Wq[n * K + k]);
+      for (int64_t k = 0; k < K; ++k) s += xd[t * K + k] * wd[n * K + k];
       acc[t * N + n] = s;
     }
   }
+  free(xd); free(wd);
 }
 
 int onext_fp8_matmul(const uint16_t* X, int64_t T, int64_t K, const uint8_t* Wq, const float* sw,

@@ -39,8 +39,8 @@ MUTANTS = {
     # FP8: the sign of zero dropped
     "e4m3_unsigned_zero": ("const uint8_t sign = signbit(x) ? 0x80 : 0;", "const uint8_t sign = (x < 0) ? 0x80 : 0;"),
     # FP8: the last product dropped
-    "fp8_gemm_drops_last_k": ("for (int64_t k = 0; k < K; ++k)\n        s += (double)onext_e4m3_to_float",
-                              "for (int64_t k = 0; k + 1 < K; ++k)\n        s += (double)onext_e4m3_to_float"),
+    "fp8_gemm_drops_last_k": ("for (int64_t k = 0; k < K; ++k) s += xd[t * K + k] * wd[n * K + k];",
+                              "for (int64_t k = 0; k + 1 < K; ++k) s += xd[t * K + k] * wd[n * K + k];"),
     # stored columns: a miss uses the raw code without its scale
     "miss_without_scale": ("onext_reconstruct_weight(Wq[n * K + k], sw[n]);",
                            "onext_reconstruct_weight(Wq[n * K + k], 1.0f);"),
