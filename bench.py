@@ -9,8 +9,11 @@ L2 is flushed (256 MiB write) before every timed step.  Metric: algorithmic
 HBM bytes / time (Wq + Wscale + outlier columns of W + X + Y).
 
 Prefill workloads (--workload 7b_prefill | 13b_up | 70b_up) report effective
-TOPS = 2 T N K / time; at N=1 they are also measured by default and reported
-under "also".
+TOPS = 2 T N K / time.  At N=1 the default run also measures, under "also":
+the prefill workloads (70B at thresholds 6, 4 and inf), the FP8 (E4M3) and
+SmoothQuant W8A8 variants on the 7B / 13B prefill shapes, and the decode step
+with E4M3 codes and with a column store of outlier weights instead of the fp16
+W; each entry with its roofline and the CPU oracle timed on a sample of it.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
@@ -177,11 +180,14 @@ REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
 
 
 class ClockSampler:
-    """Samples SM clock and throttle reasons through NVML while the timed region runs."""
+    """Samples SM clock and throttle reasons through NVML, back to back, from
+    before the timed region to its end; `mark()` opens the timed window (a
+    sample is also taken synchronously at each end of it)."""
 
-    def __init__(self, cuda_index: int, period_s: float = 0.01):
-        self.samples, self.reasons, self.max_mhz, self.ok = [], 0, None, False
+    def __init__(self, cuda_index: int, period_s: float = 0.0005):
+        self.samples, self.window, self.reasons, self.max_mhz, self.ok = [], [], 0, None, False
         self._stop = threading.Event()
+        self._in_window = False
         self._period = period_s
         try:
             import pynvml
@@ -198,15 +204,31 @@ class ClockSampler:
             self.ok = False
         self._t = threading.Thread(target=self._run, daemon=True)
 
-    def _run(self):
+    def _sample(self):
         nv = self._nv
+        try:
+            mhz = nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM)
+            r = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+        except Exception:
+            return
+        self.samples.append(mhz)
+        if self._in_window:
+            self.window.append(mhz)
+            self.reasons |= r
+
+    def _run(self):
         while not self._stop.is_set():
-            try:
-                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
-                self.reasons |= nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
-            except Exception:
-                pass
+            self._sample()
             time.sleep(self._period)
+
+    def mark(self, inside: bool):
+        if self.ok:
+            if inside:
+                self._in_window = True
+                self._sample()
+            else:
+                self._sample()
+                self._in_window = False
 
     def __enter__(self):
         if self.ok:
@@ -219,26 +241,39 @@ class ClockSampler:
             self._t.join()
 
     def summary(self) -> dict:
-        if not self.ok or not self.samples:
+        if not self.ok or not self.window:
             return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0,
                     "note": "NVML sampling unavailable"}
         names = [n for bit, n in REASONS.items() if self.reasons & bit]
-        return {"sm_mhz": float(statistics.median(self.samples)), "sm_max_mhz": self.max_mhz,
-                "reasons": names, "samples": len(self.samples)}
+        return {"sm_mhz": float(statistics.median(self.window)), "sm_max_mhz": self.max_mhz,
+                "reasons": names, "samples": len(self.window), "sm_mhz_min": float(min(self.window))}
 
 
 # ----------------------------------------------------------------- workloads
 
-class Workload:
-    """Device-resident inputs and the list of calls one step makes."""
+VARIANTS = ("llmint8", "fp8", "smoothquant", "stored")
 
-    def __init__(self, name: str, device, seed: int = 0, taus=None):
+
+class Workload:
+    """Device-resident inputs and the list of calls one step makes.
+
+    variant: "llmint8" (llmint8_matmul with the fp16 W), "fp8" (E4M3 codes,
+    llmint8_fp8_matmul), "smoothquant" (W8A8 with factors from the workload's
+    own activations at alpha 0.5, llmint8_smoothquant_matmul) or "stored"
+    (llmint8_matmul_stored with the workload's systematic outlier dims in a
+    column store and no fp16 W)."""
+
+    def __init__(self, name: str, device, seed: int = 0, taus=None, variant: str = "llmint8",
+                 prefetch_next: bool = True):
         import torch
         import int8_mixed_precision_outlier_b200 as L
-        self.L, self.name, self.device = L, name, device
+        assert variant in VARIANTS, variant
+        self.L, self.name, self.device, self.variant = L, name, device, variant
+        # decode: each call asks L2 for the next call's weight codes (the next layer)
+        self.prefetch_next = prefetch_next and name == "7b_decode" and variant == "llmint8"
         cfg = synth.WORKLOADS[name]
         self.K, self.N = cfg["K"], cfg["N"]
-        self.calls = []  # dicts: X, Wq, sw, W, Y, tau, T, host data
+        self.calls = []
         if name == "7b_decode":
             ws = L.alloc_workspace(16, self.N, self.K, device)
             for layer, T in enumerate(DECODE_TS):
@@ -249,15 +284,22 @@ class Workload:
             w = synth.workload(name, seed=seed)
             ws = L.alloc_workspace(w["T"], self.N, self.K, device)
             taus = taus if taus is not None else ((THRESHOLD,) if name != "70b_up" else w["thresholds"])
-            Wd = None
+            shared = None
             for tau in taus:
-                Wd = self._add(w, w["T"], tau, ws, share_w=Wd)
+                shared = self._add(w, w["T"], tau, ws, shared=shared)
             self.unit, self.kind = "TOPS", "tensor"
+        for i, c in enumerate(self.calls):
+            c["next_Wq"] = self.calls[i + 1]["Wq"] if self.prefetch_next and i + 1 < len(self.calls) else None
         torch.cuda.synchronize()
         self.bytes_per_step = sum(c["bytes"] for c in self.calls)
         self.ops_per_step = sum(c["ops"] for c in self.calls)
-        self.launches_per_step = sum(L.llmint8_kernel_launches(c["T"], self.N, self.K) for c in self.calls)
+        self.launches_per_step = sum(self._launches(c["T"]) for c in self.calls)
         self.graph = None
+
+    def _launches(self, T):
+        if self.variant == "smoothquant":
+            return 2                     # activation kernel + GEMV / GEMM
+        return self.L.llmint8_kernel_launches(T, self.N, self.K)
 
     def capture(self):
         """One step as a CUDA graph (the kernels keep their programmatic
@@ -272,67 +314,116 @@ class Workload:
         self.graph = g
         return g
 
-    def _add(self, w, T, tau, ws, share_w=None):
+    def _add(self, w, T, tau, ws, shared=None):
         import torch
         L = self.L
         X = torch.from_numpy(w["X"]).to(self.device)
-        if share_w is None:
-            W = torch.from_numpy(w["W"]).to(self.device)
-            Wq, sw = L.llmint8_quantize_weight(W)
-            share_w = (W, Wq, sw)
-        W, Wq, sw = share_w
-        Y = torch.empty((T, self.N), dtype=torch.float16, device=self.device)
-        _, _, idx = L.llmint8_detect_quantize(X, tau)
-        nO = int(idx.numel())
         K, N = self.K, self.N
+        if shared is None:
+            W = torch.from_numpy(w["W"]).to(self.device)
+            shared = {"W": W}
+            if self.variant == "fp8":
+                shared["Wq"], shared["sw"] = L.llmint8_fp8_quantize_weight(W)
+            elif self.variant == "smoothquant":
+                ax = L.llmint8_column_absmax(X)
+                aw = L.llmint8_column_absmax(W)
+                shared["s"] = L.llmint8_smooth_factors(ax, aw, 0.5)
+                shared["Wq"], shared["sw"] = L.llmint8_smoothquant_quantize_weight(W, shared["s"])
+                shared["ws"] = torch.empty(int(L.load_library().llmint8_smoothquant_workspace_bytes(T, K)),
+                                           dtype=torch.uint8, device=self.device)
+            else:
+                shared["Wq"], shared["sw"] = L.llmint8_quantize_weight(W)
+            if self.variant == "stored":
+                cols = torch.from_numpy(np.sort(w["dims"]).astype(np.int32)).to(self.device)
+                shared["slot"], shared["Wst"] = L.llmint8_outlier_store_build(W, cols)
+                shared["n_store"] = int(cols.numel())
+                shared["miss"] = torch.zeros(1, dtype=torch.int32, device=self.device)
+        Y = torch.empty((T, N), dtype=torch.float16, device=self.device)
+        if self.variant == "smoothquant":
+            nO = 0
+        else:
+            _, _, idx = L.llmint8_detect_quantize(X, tau)
+            nO = int(idx.numel())
         algo_bytes = N * K + 4 * N + 2 * N * nO + 2 * T * K + 2 * T * N
-        self.calls.append(dict(X=X, W=W, Wq=Wq, sw=sw, Y=Y, ws=ws, tau=tau, T=T, nO=nO,
-                               bytes=algo_bytes, ops=2 * T * N * K, host_X=w["X"], host_W=w["W"]))
-        return share_w
+        c = dict(X=X, Y=Y, ws=ws, tau=tau, T=T, nO=nO, bytes=algo_bytes, ops=2 * T * N * K,
+                 host_X=w["X"], host_W=w["W"], dims=w["dims"])
+        c.update({k: v for k, v in shared.items() if k not in ("ws",)})
+        if self.variant == "smoothquant":
+            c["ws"] = shared["ws"]
+        self.calls.append(c)
+        return shared
+
+    def call(self, c, Y=None):
+        """One library call of this workload's variant."""
+        L = self.L
+        Y = c["Y"] if Y is None else Y
+        if self.variant == "llmint8":
+            if c.get("next_Wq") is not None:
+                return L.llmint8_matmul_prefetch_next(c["X"], c["Wq"], c["sw"], c["W"], c["tau"], c["ws"], Y,
+                                                      c["next_Wq"])
+            return L.llmint8_matmul(c["X"], c["Wq"], c["sw"], c["W"], c["tau"], c["ws"], Y)
+        if self.variant == "fp8":
+            return L.llmint8_fp8_matmul(c["X"], c["Wq"], c["sw"], c["W"], c["tau"], c["ws"], Y)
+        if self.variant == "smoothquant":
+            return L.llmint8_smoothquant_matmul(c["X"], c["s"], c["Wq"], c["sw"], c["ws"], Y)
+        return L.llmint8_matmul_stored(c["X"], c["Wq"], c["sw"], c["slot"], c["Wst"], c["tau"], c["ws"], Y,
+                                       n_miss=c["miss"])
 
     def step(self):
-        L = self.L
         for c in self.calls:
-            L.llmint8_matmul(c["X"], c["Wq"], c["sw"], c["W"], c["tau"], c["ws"], c["Y"])
+            self.call(c)
 
     def metric_value(self, seconds: float, steps: int) -> float:
         if self.unit == "GB/s":
             return self.bytes_per_step * steps / seconds / 1e9
         return self.ops_per_step * steps / seconds / 1e12
 
+    def resident_weight_bytes(self) -> int:
+        """Weight bytes one call keeps on the device for its matrix."""
+        c = self.calls[0]
+        n = c["Wq"].numel() + 4 * c["sw"].numel()
+        if self.variant == "stored":
+            return n + 2 * c["Wst"].numel() + 4 * c["slot"].numel()
+        if self.variant == "smoothquant":
+            return n + 4 * self.K
+        return n + 2 * c["W"].numel()
+
 
 def time_steps(wl: Workload, steps: int, warmup: int, world: int, flush, run=None, gate_us=0.0):
-    """Events around each step on the launching stream; L2 flushed before each."""
+    """Events around each step on the launching stream; L2 flushed before each.
+    The clock sampler runs through warm-up and timing; its window is the timed
+    steps."""
     import torch
     run = run or wl.step
-    for _ in range(warmup):
-        flush.zero_(gate_us)
-        run()
     stream = torch.cuda.current_stream()
     starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
     ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
-    barrier(world)
-    torch.cuda.synchronize()
     sampler = ClockSampler(torch.cuda.current_device())
     with sampler:
+        for _ in range(warmup):
+            flush.zero_(gate_us)
+            run()
+        barrier(world)
+        torch.cuda.synchronize()
+        sampler.mark(True)
         for i in range(steps):
             flush.zero_(gate_us)
             starts[i].record(stream)
             run()
             ends[i].record(stream)
         torch.cuda.synchronize()
+        sampler.mark(False)
     barrier(world)
     total_ms = sum(s.elapsed_time(e) for s, e in zip(starts, ends))
     return total_ms, sampler.summary()
 
 
-def time_main_kernel(wl: Workload, steps: int, flush) -> tuple[float, float]:
-    """Average duration of the roofline unit on cold L2, as in the timed steps
-    (flush before each step, the step's calls in order, one launch each).
+def time_cold_units(wl: Workload, steps: int, flush) -> tuple[float, float]:
+    """Average duration of one cold unit (flush before each step, the step's
+    calls in order, one launch per event pair).
 
-    Decode: one whole call, decode_prep_kernel then gemv_kernel.  The GEMV
-    launches while the prep kernel runs and starts its weight stream then, so
-    the two share the HBM time and are timed together.  Prefill: the GEMM launch alone (events
+    Decode: one whole call (prep kernel + GEMV, which starts its weight stream
+    while the prep kernel runs).  Prefill: the GEMM launch alone (events
     between the activation kernels and it).  Returns (ms per unit, algorithmic
     bytes or ops per unit)."""
     import torch
@@ -343,9 +434,9 @@ def time_main_kernel(wl: Workload, steps: int, flush) -> tuple[float, float]:
         for c in wl.calls:
             b = torch.cuda.Event(enable_timing=True)
             e = torch.cuda.Event(enable_timing=True)
-            if wl.unit == "GB/s":
+            if wl.unit == "GB/s" or wl.variant != "llmint8":
                 b.record()
-                L.llmint8_matmul(c["X"], c["Wq"], c["sw"], c["W"], c["tau"], c["ws"], c["Y"])
+                wl.call(c)
                 e.record()
             else:
                 L.llmint8_matmul_profile(c["X"], c["Wq"], c["sw"], c["W"], c["tau"], c["ws"], c["Y"], b, e,
@@ -358,28 +449,59 @@ def time_main_kernel(wl: Workload, steps: int, flush) -> tuple[float, float]:
 
 
 def main_kernel_name(wl: Workload) -> str:
-    return "decode_call" if wl.unit == "GB/s" else "gemm_pair_kernel"
-
-
-def roofline(wl: Workload, kern_ms: float, algo_per_launch: float, peaks: dict, traffic=None) -> dict:
     if wl.unit == "GB/s":
-        achieved = algo_per_launch / (kern_ms * 1e-3) / 1e9
-        peak = peaks["hbm_gbs"]
-        return {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
-                "frac": round(achieved / peak, 4), "traffic": traffic,
-                "kernel": "decode_prep_kernel + gemv_kernel (one call; the GEMV streams the weights "
-                          "and starts that stream while the prep kernel runs)",
-                "peak_source": f"{peaks['source']} hbm_gbs (copy, burst)",
-                "frac_of_published": round(achieved / PUBLISHED["hbm_gbs"], 4),
-                "algo_bytes_per_launch": int(algo_per_launch), "ms_per_launch": round(kern_ms, 5)}
-    achieved = algo_per_launch / (kern_ms * 1e-3) / 1e12
-    peak = peaks["bf16_tflops"] * INT8_PER_BF16
-    return {"bound": "tensor", "achieved": round(achieved, 1), "peak": round(peak, 1), "unit": "TOPS",
+        return "decode_call" if wl.variant == "llmint8" else f"decode_call_{wl.variant}"
+    return "gemm_pair_kernel" if wl.variant == "llmint8" else f"call_{wl.variant}"
+
+
+def decode_roofline(wl: Workload, ms_per_step: float, cold_ms: float, cold_algo: float, peaks: dict,
+                    traffic=None) -> dict:
+    """The decode call as it runs inside the graph-replayed step: the step's
+    algorithmic bytes over its device time (5 calls per step), so that the
+    unit and the headline share one definition; the cold single call (events
+    around one call after an L2 flush) is reported beside it as a bound."""
+    achieved = wl.bytes_per_step / (ms_per_step * 1e-3) / 1e9
+    peak = peaks["hbm_gbs"]
+    cold = cold_algo / (cold_ms * 1e-3) / 1e9
+    return {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
             "frac": round(achieved / peak, 4), "traffic": traffic,
-            "kernel": "gemm_pair_kernel (persistent CTA pairs, tcgen05 cta_group::2 kind::i8 + kind::f16)",
-            "peak_source": f"{peaks['source']} bf16_tflops (burst) x 2 (nominal int8/bf16 ratio)",
+            "kernel": "decode_prep_kernel + gemv_kernel, one call as it runs in the step "
+                      f"({len(wl.calls)} calls per step; step bytes / step time"
+                      + ("; each call requests the next layer's weight codes into L2)" if wl.prefetch_next else ")"),
+            "peak_source": f"{peaks['source']} hbm_gbs (copy, burst)",
+            "frac_of_published": round(achieved / PUBLISHED["hbm_gbs"], 4),
+            "algo_bytes_per_launch": int(wl.bytes_per_step / len(wl.calls)),
+            "ms_per_launch": round(ms_per_step / len(wl.calls), 5),
+            "cold_call": {"achieved": round(cold, 1), "frac": round(cold / peak, 4), "ms": round(cold_ms, 5),
+                          "how": "one call between events after an L2 flush (a bound: no overlap with the "
+                                 "neighbouring calls)"}}
+
+
+def prefill_roofline(wl: Workload, kern_ms: float, c: dict, peaks: dict, traffic=None, kernel=None) -> dict:
+    """Tensor-bound roofline of one prefill launch.  The target time splits
+    the work as the method does: 2 T N |R| products on the 8-bit tensor peak
+    (int8 or fp8: measured bf16 burst x 2, the nominal ratio) and 2 T N |O|
+    on the fp16 peak (measured bf16 burst, the same rate).  achieved =
+    2 T N K / time; peak = 2 T N K / target time, so frac = target / time."""
+    T, N, K = c["T"], wl.N, wl.K
+    p8 = peaks["bf16_tflops"] * INT8_PER_BF16 * 1e12
+    p16 = peaks["bf16_tflops"] * 1e12
+    nO = c["nO"]
+    target_s = 2.0 * T * N * (K - nO) / p8 + 2.0 * T * N * nO / p16
+    ops = 2.0 * T * N * K
+    achieved = ops / (kern_ms * 1e-3) / 1e12
+    peak = ops / target_s / 1e12
+    names = {"llmint8": "gemm_pair_kernel (persistent CTA pairs, tcgen05 cta_group::2 kind::i8 + kind::f16)",
+             "fp8": "whole call: activation kernels + gemm_pair_kernel<fp8> (tcgen05 kind::f8f6f4 + kind::f16)",
+             "smoothquant": "whole call: smoothing quantize kernel + gemm_pair_kernel (kind::i8, no fp16 part)",
+             "stored": "whole call: activation kernels with the column-store gather + gemm_pair_kernel"}
+    return {"bound": "tensor", "achieved": round(achieved, 1), "peak": round(peak, 1), "unit": "TOPS",
+            "frac": round(achieved / peak, 4), "traffic": traffic, "kernel": kernel or names[wl.variant],
+            "peak_source": f"{peaks['source']} bf16_tflops (burst) x 2 for the 8-bit part (nominal ratio), "
+                           f"x 1 for the {nO} fp16 outlier columns",
             "frac_of_published": round(achieved / PUBLISHED["int8_tops"], 4),
-            "algo_ops_per_launch": int(algo_per_launch), "ms_per_launch": round(kern_ms, 5)}
+            "algo_ops_per_launch": int(ops), "int8_ops": int(2 * T * N * (K - nO)), "f16_flops": int(2 * T * N * nO),
+            "ms_per_launch": round(kern_ms, 5)}
 
 
 def e2e_steps(wl: Workload, steps: int, warmup: int, flush, world: int = 1) -> dict:
@@ -387,14 +509,13 @@ def e2e_steps(wl: Workload, steps: int, warmup: int, flush, world: int = 1) -> d
     Every rank runs it; the value is all ranks' units over the slowest rank's
     time, and the copy bytes are the whole job's."""
     import torch
-    L = wl.L
     hx = [torch.from_numpy(c["host_X"]).pin_memory() for c in wl.calls]
     hy = [torch.empty(c["Y"].shape, dtype=torch.float16).pin_memory() for c in wl.calls]
 
     def run():
         for c, x, y in zip(wl.calls, hx, hy):
             c["X"].copy_(x, non_blocking=True)
-            L.llmint8_matmul(c["X"], c["Wq"], c["sw"], c["W"], c["tau"], c["ws"], c["Y"])
+            wl.call(c)
             y.copy_(c["Y"], non_blocking=True)
 
     total_ms, _ = time_steps(wl, steps, warmup, world, flush, run=run)
@@ -410,46 +531,65 @@ def e2e_steps(wl: Workload, steps: int, warmup: int, flush, world: int = 1) -> d
 
 # ----------------------------------------------------------------- CPU oracle
 
-def oracle_sample(name: str, seed: int = 0):
+def oracle_sample(name: str, seed: int = 0, variant: str = "llmint8", tau: float = THRESHOLD, rows=None):
     """Oracle inputs and one step's calls, on a bounded sample of the workload.
 
     Decode: the full step (five calls).  Prefill: the first `rows` rows of X
     against the full W (detection and scales then cover those rows only).
-    """
+    Each call is (fn, args, bytes, ops) with fn an oracle function."""
     from oracle import oracle as O
+    from oracle import oracle_next as ON
     cfg = synth.WORKLOADS[name]
+
+    def prepare(X, W, tau, dims):
+        if variant == "fp8":
+            Wq, sw = ON.fp8_quantize_weight(W)
+            return ON.fp8_matmul, (X, Wq, sw, W, tau)
+        if variant == "smoothquant":
+            s = ON.smooth_factors(ON.column_absmax(X), ON.column_absmax(W), 0.5)
+            Wq, sw = ON.smooth_quantize_weight(W, s)
+            return ON.smoothquant_matmul, (X, s, Wq, sw)
+        Wq, sw = O.quantize_weight(W)
+        if variant == "stored":
+            slot, Wst = ON.make_store(W, np.sort(dims))
+            return ON.matmul_stored, (X, Wq, sw, slot, Wst, tau)
+        return O.matmul, (X, Wq, sw, W, tau)
+
     calls = []
     if name == "7b_decode":
         for layer, T in enumerate(DECODE_TS):
             w = synth.workload(name, seed=seed, T=T, layer=layer)
-            Wq, sw = O.quantize_weight(w["W"])
-            nO = int(O.compact(O.detect_outliers(w["X"], THRESHOLD)).size)
-            calls.append((w["X"], Wq, sw, w["W"], THRESHOLD,
-                          cfg["N"] * cfg["K"] + 4 * cfg["N"] + 2 * cfg["N"] * nO +
+            nO = int(O.compact(O.detect_outliers(w["X"], tau)).size)
+            fn, args = prepare(w["X"], w["W"], tau, w["dims"])
+            calls.append((fn, args, cfg["N"] * cfg["K"] + 4 * cfg["N"] + 2 * cfg["N"] * nO +
                           2 * T * cfg["K"] + 2 * T * cfg["N"], 2 * T * cfg["N"] * cfg["K"]))
         return calls, "the step's 5 calls, T=1,2,4,8,16, full N and K", "GB/s"
     w = synth.workload(name, seed=seed)
-    rows = 16 if name == "70b_up" else 32
+    if rows is None:
+        rows = 16 if name == "70b_up" else 32
+    rows = min(rows, w["T"])
     Xs = np.ascontiguousarray(w["X"][:rows])
-    Wq, sw = O.quantize_weight(w["W"])
+    fn, args = prepare(Xs, w["W"], tau, w["dims"])
     T, N, K = rows, cfg["N"], cfg["K"]
-    calls.append((Xs, Wq, sw, w["W"], THRESHOLD, 0, 2 * T * N * K))
-    return calls, f"first {rows} rows of X against the full W, tau=6 (ops scaled to those rows)", "TOPS"
+    calls.append((fn, args, 0, 2 * T * N * K))
+    what = "tau=%s" % tau if variant != "smoothquant" else "alpha=0.5, factors from these rows"
+    return calls, f"first {rows} rows of X against the full W, {what} (ops counted for those rows)", "TOPS"
 
 
 def shrink_sample(calls, frac: float):
     """The same calls on the first max(1, floor(N * frac)) output rows of W
     (rows of W are independent outputs), with the algorithmic bytes and ops
-    counted for those rows."""
+    counted for those rows.  Works on calls of oracle.matmul (X, Wq, sw, W,
+    tau) as oracle_sample builds them."""
     out = []
-    for X, Wq, sw, W, tau, nbytes, ops in calls:
+    for fn, (X, Wq, sw, W, tau), nbytes, ops in calls:
         N, K = Wq.shape
         T = X.shape[0]
         n = max(1, int(N * frac))
         if nbytes:
             n_out = (nbytes - N * K - 4 * N - 2 * T * K - 2 * T * N) // (2 * N)  # |O| of this call
             nbytes = n * K + 4 * n + 2 * n * n_out + 2 * T * K + 2 * T * n
-        out.append((X, Wq[:n], sw[:n], W[:n], tau, nbytes, 2 * T * n * K))
+        out.append((fn, (X, Wq[:n], sw[:n], W[:n], tau), nbytes, 2 * T * n * K))
     return out, n
 
 
@@ -457,15 +597,22 @@ def run_oracle(calls, unit, steps: int, budget_s: float):
     from oracle import oracle as O
     done, t0 = 0, time.perf_counter()
     while done < steps:
-        for X, Wq, sw, W, tau, _, _ in calls:
-            O.matmul(X, Wq, sw, W, tau)
+        for fn, args, _, _ in calls:
+            fn(*args)
         done += 1
         if time.perf_counter() - t0 > budget_s:
             break
     dt = time.perf_counter() - t0
-    per = sum(c[5] for c in calls) if unit == "GB/s" else sum(c[6] for c in calls)
+    per = sum(c[2] for c in calls) if unit == "GB/s" else sum(c[3] for c in calls)
     value = per * done / dt / (1e9 if unit == "GB/s" else 1e12)
     return value, done, dt, O.num_threads()
+
+
+def cpu_baseline(name: str, variant: str = "llmint8", tau: float = THRESHOLD, rows=None, budget_s: float = 15.0):
+    calls, sample, unit = oracle_sample(name, variant=variant, tau=tau, rows=rows)
+    v, done, dt, cores = run_oracle(calls, unit, 1000, budget_s)
+    return {"value": round(v, 4), "unit": unit, "cores": cores, "kind": "oracle",
+            "sample": sample + f"; {done} steps in {dt:.1f} s"}
 
 
 # ----------------------------------------------------------------- arms
@@ -518,6 +665,54 @@ def workload_config(name: str) -> dict:
     return d
 
 
+# (workload, variant, threshold): the entries of "also" at N = 1; "llmint8-noprefetch" is the
+# decode step with plain llmint8_matmul calls (no request for the next layer's weights)
+ALSO = [("7b_decode", "llmint8-noprefetch", 6.0),
+        ("7b_prefill", "llmint8", 6.0), ("13b_up", "llmint8", 6.0), ("70b_up", "llmint8", 6.0),
+        ("70b_up", "llmint8", 4.0), ("70b_up", "llmint8", float("inf")),
+        ("7b_prefill", "fp8", 6.0), ("13b_up", "fp8", 6.0), ("7b_prefill", "smoothquant", None),
+        ("13b_up", "smoothquant", None), ("7b_prefill", "stored", 6.0), ("7b_decode", "fp8", 6.0),
+        ("7b_decode", "stored", 6.0)]
+
+# oracle rows timed per prefill entry (about 1-10 s of CPU work each)
+ORACLE_ROWS = {"7b_prefill": 256, "13b_up": 128, "70b_up": 16}
+
+
+def also_entry(name, variant, tau, device, peaks, flush, steps, oracle_budget_s):
+    import torch
+    taus = None if tau is None else (tau,)
+    prefetch = not variant.endswith("-noprefetch")
+    variant = variant.replace("-noprefetch", "")
+    w2 = Workload(name, device, taus=taus, variant=variant, prefetch_next=prefetch)
+    w2.capture()
+    ms, ck = time_steps(w2, steps, 3, 1, flush, run=w2.graph.replay)
+    status = w2.L.llmint8_sync_status()
+    c = w2.calls[0]
+    entry = {"workload": name, "variant": variant if prefetch or w2.unit != "GB/s" else variant + " (no next-layer prefetch)",
+             "value": round(w2.metric_value(ms * 1e-3, steps), 2),
+             "unit": w2.unit, "ms_per_step": round(ms / steps, 4), "n_outliers": c["nO"],
+             "threshold": tau, "clocks": ck, "device_status": w2.L.llmint8_status_string(status),
+             "resident_weight_bytes": w2.resident_weight_bytes()}
+    if variant == "stored":
+        entry["store_columns"] = int(c["n_store"])
+        entry["misses_last_call"] = int(c["miss"].item())
+    if w2.unit == "GB/s":
+        cold_ms, cold_algo = time_cold_units(w2, 10, flush)
+        entry["roofline"] = decode_roofline(w2, ms / steps, cold_ms, cold_algo, peaks,
+                                            traffic=recorded_traffic(name, main_kernel_name(w2)))
+    else:
+        km, _ = time_cold_units(w2, 10, flush)
+        entry["roofline"] = prefill_roofline(w2, km, c, peaks,
+                                             traffic=recorded_traffic(name, main_kernel_name(w2)))
+        call_tops = w2.ops_per_step / (ms / steps * 1e-3) / 1e12   # the whole call, graph-replayed
+        entry["call_roofline_frac"] = round(call_tops / entry["roofline"]["peak"], 4)
+    del w2
+    torch.cuda.empty_cache()
+    entry["cpu_baseline"] = cpu_baseline(name, variant=variant, tau=THRESHOLD if tau is None else tau,
+                                         rows=ORACLE_ROWS.get(name), budget_s=oracle_budget_s)
+    return entry
+
+
 def run_ours(args):
     import torch
     rank, world, local = dist_env()
@@ -546,41 +741,30 @@ def run_ours(args):
     units = reduce_sum((wl.bytes_per_step if wl.unit == "GB/s" else wl.ops_per_step) * args.steps, world)
     value = units / (t_max * 1e-3) / (1e9 if wl.unit == "GB/s" else 1e12)
     status = L.llmint8_sync_status()
-    kern_ms, algo = time_main_kernel(wl, 10, flush)
+    cold_ms, cold_algo = time_cold_units(wl, 10, flush)
+    traffic = recorded_traffic(args.workload, main_kernel_name(wl))
+    if wl.unit == "GB/s":
+        roof = decode_roofline(wl, total_ms / args.steps, cold_ms, cold_algo, peaks, traffic=traffic)
+    else:
+        roof = prefill_roofline(wl, cold_ms, wl.calls[0], peaks, traffic=traffic)
     line = {
         "metric": METRIC, "value": round(value, 3), "unit": wl.unit, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(t_max / args.steps, 5),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int8",
         "data": "synthetic", "config": workload_config(args.workload),
-        "roofline": roofline(wl, kern_ms, algo, peaks,
-                             traffic=recorded_traffic(args.workload, main_kernel_name(wl))),
+        "roofline": roof,
         "gpu_launches": wl.launches_per_step * args.steps,
         "clocks": clocks, "device_status": L.llmint8_status_string(status),
     }
     line["e2e"] = e2e_steps(wl, args.steps, args.warmup, flush, world)  # collective: every rank
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        calls, sample, unit = oracle_sample(args.workload)
-        v, done, dt, cores = run_oracle(calls, unit, 1000, args.cpu_budget_s)
-        line["cpu_baseline"] = {"value": round(v, 4), "unit": unit, "cores": cores, "kind": "oracle",
-                                "sample": sample + f"; {done} steps in {dt:.1f} s"}
+        line["cpu_baseline"] = cpu_baseline(args.workload, budget_s=args.cpu_budget_s)
     if rank == 0 and world == 1 and args.also:
-        also = []
-        for name in ("7b_prefill", "13b_up", "70b_up"):
-            if name == args.workload:
-                continue
-            w2 = Workload(name, device, taus=(THRESHOLD,))
-            w2.capture()
-            ms, ck = time_steps(w2, args.also_steps, 3, 1, flush, run=w2.graph.replay)
-            km, ka = time_main_kernel(w2, 10, flush)
-            also.append({"workload": name, "value": round(w2.metric_value(ms * 1e-3, args.also_steps), 2),
-                         "unit": w2.unit, "ms_per_call": round(ms / args.also_steps, 4),
-                         "n_outliers": w2.calls[0]["nO"], "threshold": THRESHOLD,
-                         "roofline": roofline(w2, km, ka, peaks,
-                                              traffic=recorded_traffic(name, main_kernel_name(w2))),
-                         "sm_mhz": ck.get("sm_mhz")})
-            del w2
-            torch.cuda.empty_cache()
-        line["also"] = also
+        del wl
+        torch.cuda.empty_cache()
+        line["also"] = [also_entry(name, variant, tau, device, peaks, flush, args.also_steps, args.also_cpu_budget_s)
+                        for name, variant, tau in ALSO if not (name == args.workload and variant == "llmint8")
+                        and not (name != "7b_decode" and variant.endswith("-noprefetch"))]
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -600,6 +784,7 @@ def main(argv=None):
     ap.add_argument("--no-also", dest="also", action="store_false")
     ap.add_argument("--also-steps", type=int, default=20)
     ap.add_argument("--cpu-budget-s", type=float, default=15.0)
+    ap.add_argument("--also-cpu-budget-s", type=float, default=4.0)
     ap.add_argument("--ref-budget-s", type=float, default=120.0)
     args = ap.parse_args(argv)
     if args.warmup < 3:

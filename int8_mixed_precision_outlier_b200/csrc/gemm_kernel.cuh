@@ -13,6 +13,9 @@
 // added; '三、模型量化' (lowentro.cn) Q2/Q4: r' = s*q on both operands).
 // |O| is read from device memory, so the host never waits for it.
 //
+// FP8 (template flag): the same kernels for E4M3 codes ('量化压缩实战' §3.6),
+// the 8-bit product as tcgen05.mma kind::f8f6f4 into an f32 accumulator.
+//
 // Operands arrive by TMA (128-byte swizzle, one 128-byte K row per box row)
 // into a STAGES-deep ring; warp 0 issues the copies, warp 1 issues the MMAs
 // and owns TMEM, warps 2-5 run the epilogue.  Every mbarrier wait is bounded.
@@ -46,7 +49,7 @@ struct Params {
   const float* sw;
   const int32_t* n_out;
   uint16_t* Y;
-  int32_t* acc_out;  // optional int32 [T][N]
+  int32_t* acc_out;  // optional int32 [T][N] (FP8: the f32 accumulator's bits)
   uint64_t wait_ns;
 };
 
@@ -58,14 +61,15 @@ struct Params {
 // there are outlier columns.  The tile's sw values are staged in shared memory
 // (sw_s, BN floats) while the MMAs still run, so that draining TMEM waits on
 // no global load; then it waits (bounded) for `tfull`.
+template <bool FP8>
 __device__ __forceinline__ void epilogue_rows(const Params& p, uint32_t tmem_base, int q, int lane, int etid,
                                               int m0, int n0, uint64_t* tfull, float* sw_s) {
-  for (int j = etid; j < BN; j += 128) sw_s[j] = n0 + j < p.N ? __ldg(p.sw + n0 + j) : 0.0f;
+  for (int j = etid; j < BN; j += 128) sw_s[j] = (p.Y && n0 + j < p.N) ? __ldg(p.sw + n0 + j) : 0.0f;
   named_barrier(1, 128);
   const int row = m0 + q * 32 + lane;
-  const int nO = *p.n_out;
+  const int nO = load_count(p.n_out);
   const bool has_o = nO > 0;
-  const float sxr = row < p.T ? p.sx[row] : 0.0f;
+  const float sxr = (p.Y && row < p.T) ? p.sx[row] : 0.0f;
   const bool ok = mbar_wait(tfull, 0, p.wait_ns, kErrTimeoutEpilogue);
   if (!__all_sync(0xffffffffu, ok)) return;  // warp-uniform before the .sync.aligned loads
   tc_fence_after();
@@ -86,22 +90,23 @@ __device__ __forceinline__ void epilogue_rows(const Params& p, uint32_t tmem_bas
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
           const float swn = sw_s[cc + j + h];
-          y[h] = static_cast<float>(static_cast<int32_t>(ra[j + h])) * sxr * swn +
-                 (has_o ? __uint_as_float(rb[j + h]) : 0.0f);
+          y[h] = acc_value<FP8>(ra[j + h]) * sxr * swn + (has_o ? __uint_as_float(rb[j + h]) : 0.0f);
         }
         packed[j >> 1] = static_cast<uint32_t>(__half_as_ushort(__float2half_rn(y[0]))) |
                          (static_cast<uint32_t>(__half_as_ushort(__float2half_rn(y[1]))) << 16);
       }
-      uint16_t* yrow = p.Y + static_cast<int64_t>(row) * p.N + nbase;
-      if (vec_ok && nbase + 32 <= p.N) {
-        uint4* dst = reinterpret_cast<uint4*>(yrow);
+      if (p.Y) {
+        uint16_t* yrow = p.Y + static_cast<int64_t>(row) * p.N + nbase;
+        if (vec_ok && nbase + 32 <= p.N) {
+          uint4* dst = reinterpret_cast<uint4*>(yrow);
 #pragma unroll
-        for (int v = 0; v < 4; ++v)
-          dst[v] = make_uint4(packed[4 * v], packed[4 * v + 1], packed[4 * v + 2], packed[4 * v + 3]);
-      } else {
+          for (int v = 0; v < 4; ++v)
+            dst[v] = make_uint4(packed[4 * v], packed[4 * v + 1], packed[4 * v + 2], packed[4 * v + 3]);
+        } else {
 #pragma unroll
-        for (int j = 0; j < 32; ++j)
-          if (nbase + j < p.N) yrow[j] = static_cast<uint16_t>(packed[j >> 1] >> ((j & 1) * 16));
+          for (int j = 0; j < 32; ++j)
+            if (nbase + j < p.N) yrow[j] = static_cast<uint16_t>(packed[j >> 1] >> ((j & 1) * 16));
+        }
       }
       if (p.acc_out) {
         int32_t* arow = p.acc_out + static_cast<int64_t>(row) * p.N + nbase;
@@ -113,6 +118,7 @@ __device__ __forceinline__ void epilogue_rows(const Params& p, uint32_t tmem_bas
   }
 }
 
+template <bool FP8>
 __global__ void __launch_bounds__(THREADS, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmap_xq, const __grid_constant__ CUtensorMap tmap_wq,
                 const __grid_constant__ CUtensorMap tmap_xo, const __grid_constant__ CUtensorMap tmap_wo,
@@ -172,7 +178,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
       pdl_wait();
       for (int i = 0; i < pre; ++i) tma_load_2d(stage_a(i), &tmap_xq, &full[i], i * BK, m0);
-      const int nO = *p.n_out;
+      const int nO = load_count(p.n_out);
       const int OB = (nO + 63) / 64;
       const int total = KB + OB;
       int issued = pre;
@@ -197,10 +203,10 @@ __global__ void __launch_bounds__(THREADS, 1)
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       pdl_wait();
-      const int nO = *p.n_out;
+      const int nO = load_count(p.n_out);
       const int OB = (nO + 63) / 64;
       const int total = p.KB + OB;
-      constexpr uint32_t idesc_i = idesc_i8_s32(BM, BN);
+      constexpr uint32_t idesc_i = idesc_codes<FP8>(BM, BN);
       constexpr uint32_t idesc_h = idesc_f16_f32(BM, BN);
       const uint32_t d_acc = tmem_base;
       const uint32_t d_yo = tmem_base + BN;
@@ -215,8 +221,8 @@ __global__ void __launch_bounds__(THREADS, 1)
         if (i < p.KB) {
 #pragma unroll
           for (int k = 0; k < BK / 32; ++k)
-            mma_i8(d_acc, make_sdesc_k_sw128(a0 + k * 32), make_sdesc_k_sw128(b0 + k * 32), idesc_i,
-                   (i > 0 || k > 0) ? 1u : 0u);
+            mma_codes<FP8>(d_acc, make_sdesc_k_sw128(a0 + k * 32), make_sdesc_k_sw128(b0 + k * 32), idesc_i,
+                           (i > 0 || k > 0) ? 1u : 0u);
         } else {
 #pragma unroll
           for (int k = 0; k < BK / 32; ++k)
@@ -232,8 +238,8 @@ __global__ void __launch_bounds__(THREADS, 1)
   } else {
     // ------------------------------------------------------------ epilogue
     pdl_wait();
-    epilogue_rows(p, tmem_base, warp & 3, lane, static_cast<int>(threadIdx.x) - 64, m0, n0, tfull,
-                  reinterpret_cast<float*>(smem + STAGES * STAGE_BYTES + 256));
+    epilogue_rows<FP8>(p, tmem_base, warp & 3, lane, static_cast<int>(threadIdx.x) - 64, m0, n0, tfull,
+                       reinterpret_cast<float*>(smem + STAGES * STAGE_BYTES + 256));
   }
 
   // Lane 0 of warps 0 and 1 ran a role loop alone: bring each warp back
@@ -289,6 +295,7 @@ __device__ __forceinline__ void pair_tile(const Params& p, int tile, uint32_t ra
 }
 
 // 32 outputs of one row: y = fp16(acc * sxr * sw + yo), packed in pairs.
+template <bool FP8>
 __device__ __forceinline__ void dequant32(const uint32_t (&ra)[32], const uint32_t (&rb)[32], bool has_o, float sxr,
                                           const float* sw32, uint32_t (&packed)[16]) {
 #pragma unroll
@@ -296,13 +303,13 @@ __device__ __forceinline__ void dequant32(const uint32_t (&ra)[32], const uint32
     float y[2];
 #pragma unroll
     for (int h = 0; h < 2; ++h)
-      y[h] = static_cast<float>(static_cast<int32_t>(ra[j + h])) * sxr * sw32[j + h] +
-             (has_o ? __uint_as_float(rb[j + h]) : 0.0f);
+      y[h] = acc_value<FP8>(ra[j + h]) * sxr * sw32[j + h] + (has_o ? __uint_as_float(rb[j + h]) : 0.0f);
     const __half2 h2 = __floats2half2_rn(y[0], y[1]);  // y[0] in the low half
     packed[j >> 1] = *reinterpret_cast<const uint32_t*>(&h2);
   }
 }
 
+template <bool FP8>
 __global__ void __launch_bounds__(P_THREADS, 1)
     gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_xq, const __grid_constant__ CUtensorMap tmap_wq,
                      const __grid_constant__ CUtensorMap tmap_xo, const __grid_constant__ CUtensorMap tmap_wo,
@@ -373,7 +380,7 @@ __global__ void __launch_bounds__(P_THREADS, 1)
       }
       pdl_wait();
       for (int i = 0; i < pre; ++i) tma_load_2d_pair(stage_a(i), &tmap_xq, full_of(i), i * BK, m0);
-      const int total = KB + (*p.n_out + 63) / 64;
+      const int total = KB + (load_count(p.n_out) + 63) / 64;
       int it = pre;  // k-blocks issued so far, over all tiles: stage it % P_STAGES
       int kb = pre;
       bool ok = true;
@@ -405,8 +412,8 @@ __global__ void __launch_bounds__(P_THREADS, 1)
     // ------------------------------------------------------------ MMA issuer (even CTA)
     if (lane == 0 && rank == 0) {
       pdl_wait();
-      const int total = p.KB + (*p.n_out + 63) / 64;
-      const uint32_t idesc_i = idesc_i8_s32(2 * BM, p.bn);
+      const int total = p.KB + (load_count(p.n_out) + 63) / 64;
+      const uint32_t idesc_i = idesc_codes<FP8>(2 * BM, p.bn);
       const uint32_t idesc_h = idesc_f16_f32(2 * BM, p.bn);
       const uint32_t d_acc = tmem_base;
       const uint32_t d_yo = tmem_base + static_cast<uint32_t>(p.bn);
@@ -428,8 +435,8 @@ __global__ void __launch_bounds__(P_THREADS, 1)
           if (kb < p.KB) {
 #pragma unroll
             for (int k = 0; k < BK / 32; ++k)
-              mma_i8_pair(d_acc, make_sdesc_k_sw128(a0 + k * 32), make_sdesc_k_sw128(b0 + k * 32), idesc_i,
-                          (kb > 0 || k > 0) ? 1u : 0u);
+              mma_codes_pair<FP8>(d_acc, make_sdesc_k_sw128(a0 + k * 32), make_sdesc_k_sw128(b0 + k * 32),
+                                  idesc_i, (kb > 0 || k > 0) ? 1u : 0u);
           } else {
 #pragma unroll
             for (int k = 0; k < BK / 32; ++k)
@@ -454,7 +461,7 @@ __global__ void __launch_bounds__(P_THREADS, 1)
     const int r_loc = q * 32 + lane;                           // row within this CTA's 128
     uint8_t* yb = ybuf + set * P_YBUF_BYTES;                   // this set's staging box
     pdl_wait();
-    const bool has_o = *p.n_out > 0;
+    const bool has_o = load_count(p.n_out) > 0;
     const uint32_t tempty_lead = map_shared_rank(tempty, 0);
     const uint32_t lane_addr = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
     const uint32_t yo_col = static_cast<uint32_t>(p.bn);
@@ -465,10 +472,11 @@ __global__ void __launch_bounds__(P_THREADS, 1)
       int m0, n0;
       pair_tile(p, tile, rank, &m0, &n0);
       named_barrier(5, 2 * 128);  // both sets are past the previous tile's reads of sw_s
-      for (int j = etid; j < p.bn; j += 2 * 128) sw_s[j] = n0 + j < p.N ? __ldg(p.sw + n0 + j) : 0.0f;
+      for (int j = etid; j < p.bn; j += 2 * 128)
+        sw_s[j] = (p.Y && n0 + j < p.N) ? __ldg(p.sw + n0 + j) : 0.0f;
       named_barrier(5, 2 * 128);
       const int row = m0 + r_loc;
-      const float sxr = row < p.T ? p.sx[row] : 0.0f;
+      const float sxr = (p.Y && row < p.T) ? p.sx[row] : 0.0f;
       const bool okw = mbar_wait(tfull, tc & 1, p.wait_ns, kErrTimeoutEpilogue);
       if (!named_barrier_and(2, 2 * 128, okw)) break;  // all 256 epilogue threads leave together
       tc_fence_after();
@@ -508,7 +516,7 @@ __global__ void __launch_bounds__(P_THREADS, 1)
         auto half = [&](int h, const uint32_t (&ra)[32], const uint32_t (&rb)[32]) {
           const int c0 = g * P_YCOLS + h * 32;
           uint32_t packed[16];
-          dequant32(ra, rb, has_o, sxr, sw_s + c0, packed);
+          dequant32<FP8>(ra, rb, has_o, sxr, sw_s + c0, packed);
           if (staged) {
             // 128-byte swizzle, as the store's tensor map expects: 16-byte
             // chunk c of a row sits at chunk c ^ (row % 8).
@@ -519,7 +527,7 @@ __global__ void __launch_bounds__(P_THREADS, 1)
               *reinterpret_cast<uint4*>(rowp + ((c ^ (r_loc & 7)) << 4)) =
                   make_uint4(packed[4 * v], packed[4 * v + 1], packed[4 * v + 2], packed[4 * v + 3]);
             }
-          } else if (!p.y_tma && row < p.T) {
+          } else if (!p.y_tma && p.Y && row < p.T) {
             const int nbase = n0 + c0;
             uint16_t* yrow = p.Y + static_cast<int64_t>(row) * p.N + nbase;
             if (vec_ok && nbase + 32 <= p.N) {

@@ -60,7 +60,7 @@ constexpr int THREADS = 192;
 constexpr int TMEM_COLS = 32;              // 2 accumulators x 16 columns
 constexpr int XO_CHUNK = 64;               // outlier columns staged per epilogue pass
 constexpr int SMEM_BYTES = 1024 /*alignment slack*/ + STAGES * STAGE_BYTES + 256 +
-                           NT * XO_CHUNK * 4 + XO_CHUNK * 4;
+                           NT * XO_CHUNK * 4 + 2 * XO_CHUNK * 4;
 
 struct Params {
   int T, N, K;
@@ -73,30 +73,56 @@ struct Params {
   const float* sx;
   const float* sw;
   const uint16_t* X;
-  const uint16_t* W;
+  const uint16_t* W;       // fp16 weight, read at the outlier columns; null with a column store
+  const int32_t* slot;     // column store: slot[k] = row of Wst holding column k, or -1
+  const uint16_t* Wst;     // column store: fp16 [n_store][N], one column of W per row
+  const int8_t* Wqr;       // the int8 codes, read for outlier columns missing from the store
+  int32_t* n_miss;         // optional: outlier columns missing from the store (written by CTA 0)
   const int32_t* idx;
   const int32_t* n_out;
   uint16_t* Y;
-  int32_t* acc_out;   // optional int32 [T][N]
+  int32_t* acc_out;   // optional int32 [T][N] (FP8: the f32 accumulator's bits)
+  const uint8_t* pf_next;  // optional: bytes to request into L2 for the call that follows
+  int64_t pf_bytes;        // (a multiple of 16; CTA c takes the c-th equal share)
   uint64_t wait_ns;
 };
+
+// The fp16 weight W[n, k] of an outlier column: from the fp16 weight, or from
+// the column store (slot >= 0: contiguous in n across the warp's lanes), or,
+// for a column missing from the store, fp16(fl(sw[n] * Wq[n,k])) -- the fp16
+// value of its int8 weight ('LLM quantization, part 2' (hncyxsy.com) §2.1
+// keeps outlier weights in fp16; §2.2: only 8-bit weights are kept in memory).
+__device__ __forceinline__ uint16_t outlier_weight(const Params& p, int n, int k, int slot, float swn) {
+  if (p.W) return __ldg(p.W + static_cast<int64_t>(n) * p.K + k);
+  if (slot >= 0) return __ldg(p.Wst + static_cast<int64_t>(slot) * p.N + n);
+  const float q = static_cast<float>(p.Wqr[static_cast<int64_t>(n) * p.K + k]);
+  return __half_as_ushort(__float2half_rn(__fmul_rn(swn, q)));
+}
 
 // Outlier products of output row n (all 128 epilogue threads call this
 // together, each with its own n; n >= N gives zeros):
 //   yo[t] = sum_{j<|O|} X[t, O_j] * W[n, O_j]   (fp32, ascending j), t < TMAX.
-// Per 64 outlier columns: the indices go to shared memory, then the X values
-// and the row's W values are gathered with all loads in flight at once.
+// Per 64 outlier columns: the indices (and their store slots) go to shared
+// memory, then the X values and the row's W values are gathered with all
+// loads in flight at once.
 template <int TMAX>
 __device__ __forceinline__ void outlier_products(const Params& p, int nO, int n, int etid, float* xo_s,
-                                                 int32_t* idx_s, float (&yo)[TMAX]) {
+                                                 int32_t* idx_s, int32_t* slot_s, float (&yo)[TMAX]) {
 #pragma unroll
   for (int t = 0; t < TMAX; ++t) yo[t] = 0.0f;
   const bool valid = n < p.N;
-  const uint16_t* wrow = p.W + static_cast<int64_t>(valid ? n : 0) * p.K;
+  const int nv = valid ? n : 0;
+  // The scale is read only to rebuild weights a column store does not hold
+  // (calls without outlier columns may pass no scales at all).
+  const float swn = (nO > 0 && p.slot && valid) ? p.sw[nv] : 0.0f;
   for (int j0 = 0; j0 < nO; j0 += XO_CHUNK) {
     const int cnt = min(XO_CHUNK, nO - j0);
     named_barrier(1, 128);  // the previous chunk has been read
-    if (etid < XO_CHUNK) idx_s[etid] = etid < cnt ? p.idx[j0 + etid] : 0;
+    if (etid < XO_CHUNK) {
+      const int k = etid < cnt ? p.idx[j0 + etid] : 0;
+      idx_s[etid] = k;
+      slot_s[etid] = p.slot ? p.slot[k] : -1;
+    }
     named_barrier(1, 128);
     constexpr int PER = (TMAX * XO_CHUNK + 127) / 128;
     float v[PER];
@@ -111,7 +137,8 @@ __device__ __forceinline__ void outlier_products(const Params& p, int nO, int n,
     constexpr int G = 8;  // outlier columns per batch of weight loads
     uint16_t w[G];
 #pragma unroll
-    for (int u = 0; u < G; ++u) w[u] = (valid && u < cnt) ? __ldg(wrow + idx_s[u]) : uint16_t(0);
+    for (int u = 0; u < G; ++u)
+      w[u] = (valid && u < cnt) ? outlier_weight(p, nv, idx_s[u], slot_s[u], swn) : uint16_t(0);
 #pragma unroll
     for (int i = 0; i < PER; ++i)
       if (etid + 128 * i < TMAX * XO_CHUNK) xo_s[etid + 128 * i] = v[i];
@@ -120,7 +147,8 @@ __device__ __forceinline__ void outlier_products(const Params& p, int nO, int n,
       if (jj0 > 0) {
 #pragma unroll
         for (int u = 0; u < G; ++u)
-          w[u] = (valid && jj0 + u < cnt) ? __ldg(wrow + idx_s[jj0 + u]) : uint16_t(0);
+          w[u] = (valid && jj0 + u < cnt) ? outlier_weight(p, nv, idx_s[jj0 + u], slot_s[jj0 + u], swn)
+                                          : uint16_t(0);
       }
 #pragma unroll
       for (int u = 0; u < G; ++u) {
@@ -133,8 +161,9 @@ __device__ __forceinline__ void outlier_products(const Params& p, int nO, int n,
 }
 
 // TMAX: T rounded up to a power of two (1, 2, 4, 8 or 16); the per-token
-// registers and loops of the epilogue are sized by it.
-template <int TMAX>
+// registers and loops of the epilogue are sized by it.  FP8: E4M3 codes, the
+// product as kind::f8f6f4 into an f32 accumulator ('量化压缩实战' §3.6).
+template <int TMAX, bool FP8>
 __global__ void __launch_bounds__(THREADS, 1)
     gemv_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_x,
                 const Params p) {
@@ -150,6 +179,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
   float* xo_s = reinterpret_cast<float*>(smem + STAGES * STAGE_BYTES + 256);  // [NT][XO_CHUNK]
   int32_t* idx_s = reinterpret_cast<int32_t*>(xo_s + NT * XO_CHUNK);          // [XO_CHUNK]
+  int32_t* slot_s = idx_s + XO_CHUNK;                                          // [XO_CHUNK]
 
   const int warp = static_cast<int>(warp_id());
   const int lane = static_cast<int>(lane_id());
@@ -225,6 +255,18 @@ __global__ void __launch_bounds__(THREADS, 1)
         load_b(i, s);
         ++issued;
       }
+      // Every copy of this call is requested: ask L2 for this CTA's share of
+      // the weights of the call that follows (the next layer), so that HBM
+      // keeps streaming through this call's tail and the next call's prep.
+      if (p.pf_next) {
+        const int64_t per = ((p.pf_bytes + gridDim.x - 1) / gridDim.x + 15) / 16 * 16;
+        const int64_t beg = per * blockIdx.x;
+        const int64_t end = beg + per < p.pf_bytes ? beg + per : p.pf_bytes;
+        for (int64_t a = beg; a < end; a += 32768) {
+          const int64_t sz = end - a < 32768 ? end - a : 32768;
+          bulk_prefetch_l2(p.pf_next + a, static_cast<uint32_t>(sz));
+        }
+      }
       // Leave no copy in flight: wait for the last loads of every stage.
       for (int i = issued - STAGES < 0 ? 0 : issued - STAGES; i < issued; ++i)
         mbar_wait(&full[i % STAGES], (i / STAGES) & 1, p.wait_ns, kErrTimeoutProducer);
@@ -232,7 +274,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      constexpr uint32_t idesc = idesc_i8_s32(BM, NT);
+      constexpr uint32_t idesc = idesc_codes<FP8>(BM, NT);
       int i = 0;
       bool ok = true;
       for (int c = 0; c < p.CH && ok; ++c) {
@@ -256,8 +298,8 @@ __global__ void __launch_bounds__(THREADS, 1)
             const uint32_t b0 = smem_addr(stage_b(s)) + static_cast<uint32_t>(j * B_TILE);
 #pragma unroll
             for (int k = 0; k < BK / 32; ++k)
-              mma_i8(d, make_sdesc_k_sw128(a0 + k * 32), make_sdesc_k_sw128(b0 + k * 32), idesc,
-                     (ku > 0 || j > 0 || k > 0) ? 1u : 0u);
+              mma_codes<FP8>(d, make_sdesc_k_sw128(a0 + k * 32), make_sdesc_k_sw128(b0 + k * 32), idesc,
+                             (ku > 0 || j > 0 || k > 0) ? 1u : 0u);
           }
           mma_commit(&empty[s]);
         }
@@ -273,18 +315,23 @@ __global__ void __launch_bounds__(THREADS, 1)
     const int q = warp & 3;                  // TMEM lane quadrant of this warp
     const int row = q * 32 + lane;           // chunk row = TMEM lane
     const int etid = threadIdx.x - 64;       // 0..127
-    const int nO = *p.n_out;
+    const int nO = load_count(p.n_out);
     const int T = p.T;
+    if (p.n_miss && blockIdx.x == 0 && etid == 0) {
+      int miss = 0;
+      for (int j = 0; j < nO; ++j) miss += p.slot[p.idx[j]] < 0 ? 1 : 0;
+      *p.n_miss = miss;
+    }
     float sxr[TMAX];
 #pragma unroll
-    for (int t = 0; t < TMAX; ++t) sxr[t] = t < T ? p.sx[t] : 0.0f;
+    for (int t = 0; t < TMAX; ++t) sxr[t] = (p.Y && t < T) ? p.sx[t] : 0.0f;
     for (int c = 0; c < p.CH; ++c) {
       // This row's output channel; lanes past the chunk's H rows hold none.
       const int n = row < p.H ? row0 + c * p.H + row : p.N;
       // The outlier product does not depend on the int8 accumulator: it is
       // computed while the chunk's weights stream.
       float yo[TMAX];
-      outlier_products<TMAX>(p, nO, n, etid, xo_s, idx_s, yo);
+      outlier_products<TMAX>(p, nO, n, etid, xo_s, idx_s, slot_s, yo);
       const int buf = c & 1;
       // All 128 epilogue threads agree on the outcome before going on, so a
       // timeout can never leave some of them at a named barrier.
@@ -299,14 +346,13 @@ __global__ void __launch_bounds__(THREADS, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&tempty[buf]);
       if (n < p.N) {
-        const float swn = p.sw[n];
+        const float swn = p.Y ? p.sw[n] : 0.0f;
 #pragma unroll
         for (int t = 0; t < TMAX; ++t) {
           if (t < T) {
-            const int32_t acc = static_cast<int32_t>(r[t]);
-            const float y = static_cast<float>(acc) * sxr[t] * swn + yo[t];
-            p.Y[static_cast<int64_t>(t) * p.N + n] = __half_as_ushort(__float2half_rn(y));
-            if (p.acc_out) p.acc_out[static_cast<int64_t>(t) * p.N + n] = acc;
+            const float y = acc_value<FP8>(r[t]) * sxr[t] * swn + yo[t];
+            if (p.Y) p.Y[static_cast<int64_t>(t) * p.N + n] = __half_as_ushort(__float2half_rn(y));
+            if (p.acc_out) p.acc_out[static_cast<int64_t>(t) * p.N + n] = static_cast<int32_t>(r[t]);
           }
         }
       }

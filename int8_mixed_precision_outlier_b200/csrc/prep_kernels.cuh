@@ -66,6 +66,8 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* scratch, int* to
 // ---------------------------------------------------------------------------
 // a0: per-output-channel weight quantisation, one CTA per row of W.
 // ---------------------------------------------------------------------------
+// FP8: the same with E4M3 codes and s = amax / 448.
+template <bool FP8>
 __global__ void __launch_bounds__(kPrepThreads) quantize_weight_kernel(
     const uint16_t* __restrict__ W, int K, int8_t* __restrict__ Wq, float* __restrict__ Wscale) {
   __shared__ float red[32];
@@ -75,11 +77,11 @@ __global__ void __launch_bounds__(kPrepThreads) quantize_weight_kernel(
   float m = 0.0f;
   for (int c = threadIdx.x; c < nchunk; c += blockDim.x) m = absmax8(__ldg(row + c), 0u, m);
   const float amax = block_max(m, red);
-  const float s = __fdiv_rn(amax, 127.0f);
+  const float s = __fdiv_rn(amax, code_max<FP8>());
   const float inv = scale_reciprocal(s);
   if (threadIdx.x == 0) Wscale[n] = s;
   uint2* out = reinterpret_cast<uint2*>(Wq + n * K);
-  for (int c = threadIdx.x; c < nchunk; c += blockDim.x) out[c] = quant8(__ldg(row + c), s, inv, 0u);
+  for (int c = threadIdx.x; c < nchunk; c += blockDim.x) out[c] = quant8_codes<FP8>(__ldg(row + c), s, inv, 0u);
 }
 
 // ---------------------------------------------------------------------------
@@ -191,9 +193,11 @@ __global__ void __launch_bounds__(kCompactThreads) compact_kernel(
 // The row is read with 4 loads in flight per thread for its absmax, then
 // again (from L1, where this CTA just put it) for its codes.
 // Opad = |O| rounded up to 64 (one 128-byte fp16 K block of the outlier GEMM).
+// FP8: E4M3 codes with sx = amax / 448 instead of int8 codes with amax / 127.
 // ---------------------------------------------------------------------------
 constexpr int kQuantThreads = 128;
 constexpr int kWoRowsPerCta = 8;
+constexpr int kStoreRowsPerCta = 64;  // column-store gather: 64 rows x 64 columns per tile
 constexpr int kGatherIdxCap = 1024;  // outlier indices staged in shared memory per gather CTA
 
 __device__ __forceinline__ float block128_max(float v, float* red) {
@@ -204,18 +208,63 @@ __device__ __forceinline__ float block128_max(float v, float* red) {
   return r;
 }
 
+// Outlier weights from a column store instead of the fp16 weight (W null,
+// slot / Wst set): gather CTAs take 64 rows of Wo each and walk the outlier
+// columns 64 at a time through a shared-memory tile, reading 64 consecutive
+// rows of a stored column (128 contiguous bytes) and writing 64 consecutive
+// columns of Wo.  A column missing from the store gets fp16(fl(sw[n] *
+// Wq[n,k])); CTA 0 counts those misses into *n_miss.
+struct ColumnStore {
+  const int32_t* slot = nullptr;   // [K]: row of Wst holding column k, or -1
+  const uint16_t* Wst = nullptr;   // fp16 [n_store][N]
+  const int8_t* Wq = nullptr;      // int8 codes [N][K]
+  const float* sw = nullptr;       // weight scales [N]
+  int32_t* n_miss = nullptr;       // optional
+};
+
+template <bool FP8>
 __global__ void __launch_bounds__(kQuantThreads) quant_gather_kernel(
     const uint16_t* __restrict__ X, int T, int K, const uint16_t* __restrict__ W, int N,
     const uint32_t* __restrict__ flags, const int32_t* __restrict__ idx,
     const int32_t* __restrict__ n_out, int8_t* __restrict__ Xq, float* __restrict__ sx,
-    uint16_t* __restrict__ Xo, uint16_t* __restrict__ Wo, int ldo, int gather_ctas) {
+    uint16_t* __restrict__ Xo, uint16_t* __restrict__ Wo, int ldo, int gather_ctas, const ColumnStore cs) {
   __shared__ int32_t si[kGatherIdxCap];
   __shared__ float red[4];
+  __shared__ uint16_t tile[kStoreRowsPerCta][64 + 2];
   // No early trigger: the GEMM that follows takes a whole SM's shared memory
   // per CTA, so it launches only as this kernel's CTAs complete.
   pdl_wait();
   const int nO = *n_out;
   const int opad = (nO + 63) & ~63;
+  if (static_cast<int>(blockIdx.x) < gather_ctas && !W) {
+    if (blockIdx.x == 0 && threadIdx.x == 0 && cs.n_miss) {
+      int miss = 0;
+      for (int j = 0; j < nO; ++j) miss += cs.slot[idx[j]] < 0 ? 1 : 0;
+      *cs.n_miss = miss;
+    }
+    const int n0 = static_cast<int>(blockIdx.x) * kStoreRowsPerCta;
+    const int rows = min(kStoreRowsPerCta, N - n0);
+    for (int j0 = 0; j0 < opad; j0 += 64) {
+      for (int e = threadIdx.x; e < kStoreRowsPerCta * 64; e += kQuantThreads) {
+        const int jj = e / kStoreRowsPerCta, r = e % kStoreRowsPerCta, j = j0 + jj;
+        uint16_t v = 0;
+        if (j < nO && r < rows) {
+          const int k = idx[j], sl = cs.slot[k], n = n0 + r;
+          v = sl >= 0 ? __ldg(cs.Wst + static_cast<int64_t>(sl) * N + n)
+                      : __half_as_ushort(__float2half_rn(
+                            __fmul_rn(cs.sw[n], static_cast<float>(cs.Wq[static_cast<int64_t>(n) * K + k]))));
+        }
+        tile[r][jj] = v;
+      }
+      __syncthreads();
+      for (int e = threadIdx.x; e < kStoreRowsPerCta * 64; e += kQuantThreads) {
+        const int r = e / 64, jj = e % 64;
+        if (r < rows) Wo[static_cast<int64_t>(n0 + r) * ldo + j0 + jj] = tile[r][jj];
+      }
+      __syncthreads();
+    }
+    return;
+  }
   if (static_cast<int>(blockIdx.x) < gather_ctas) {
     const int nstage = nO < kGatherIdxCap ? nO : kGatherIdxCap;
     for (int j = threadIdx.x; j < nstage; j += blockDim.x) si[j] = idx[j];
@@ -266,7 +315,7 @@ __global__ void __launch_bounds__(kQuantThreads) quant_gather_kernel(
 #pragma unroll
     for (int u = 0; u < U; ++u) m = absmax8(v[u], f[u], m);
   }
-  const float s = __fdiv_rn(block128_max(m, red), 127.0f);
+  const float s = __fdiv_rn(block128_max(m, red), code_max<FP8>());
   const float inv = scale_reciprocal(s);
   if (threadIdx.x == 0) sx[t] = s;
   // second pass: the row was just read by this CTA and is still in L1
@@ -282,7 +331,7 @@ __global__ void __launch_bounds__(kQuantThreads) quant_gather_kernel(
 #pragma unroll
     for (int u = 0; u < U; ++u) {
       const int c = c0 + kQuantThreads * u;
-      if (c < nchunk) out[c] = quant8(v[u], s, inv, f[u]);
+      if (c < nchunk) out[c] = quant8_codes<FP8>(v[u], s, inv, f[u]);
     }
   }
   for (int j = threadIdx.x; j < opad; j += kQuantThreads)
@@ -302,6 +351,7 @@ __global__ void __launch_bounds__(kQuantThreads) quant_gather_kernel(
 //     list from its own copies
 //   then: this CTA's outlier indices; codes (values kept in registers, or X
 //     re-read from L2) -> Xq
+// FP8: E4M3 codes with sx = amax / 448 instead of int8 codes with amax / 127.
 // 256 threads and at most 64 registers per CTA let a CTA share an SM with a
 // GEMV CTA, so the cluster launches while the previous call's GEMV runs.  It
 // waits for its predecessor before touching memory and lets the GEMV launch at
@@ -312,7 +362,7 @@ constexpr int kDecodeThreads = 256;
 constexpr int kDecodeInFlight = 4;   // loads per thread per round
 constexpr int kDecodeMaxSlice = 65536 / 8 / kDecodeCtas;  // chunks per CTA at K = 65536
 
-template <int TMAX>
+template <int TMAX, bool FP8>
 __global__ void __launch_bounds__(kDecodeThreads, 4) decode_prep_kernel(
     const uint16_t* __restrict__ X, int T, int K, float tau, int8_t* __restrict__ Xq,
     float* __restrict__ sx, int32_t* __restrict__ idx, int32_t* __restrict__ n_out) {
@@ -396,7 +446,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 4) decode_prep_kernel(
     float mm = 0.0f;
 #pragma unroll
     for (int r = 0; r < kDecodeCtas; ++r) mm = fmaxf(mm, part[r][tid]);
-    const float s = __fdiv_rn(mm, 127.0f);
+    const float s = __fdiv_rn(mm, code_max<FP8>());
     s_sx[tid] = s;
     s_inv[tid] = scale_reciprocal(s);
     if (rank == 0 && tid < T) sx[tid] = s;
@@ -437,9 +487,32 @@ __global__ void __launch_bounds__(kDecodeThreads, 4) decode_prep_kernel(
       const int e = base + u * kDecodeThreads;
       if (e < items && t < T) {
         const int c = e / TMAX;
-        reinterpret_cast<uint2*>(Xq + static_cast<int64_t>(t) * K)[c_begin + c] = quant8(v[u], st, it, fm[c]);
+        reinterpret_cast<uint2*>(Xq + static_cast<int64_t>(t) * K)[c_begin + c] =
+            quant8_codes<FP8>(v[u], st, it, fm[c]);
       }
     }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Column store build (offline): Wst[i][n] = W[n, cols[i]] and slot[cols[i]] = i
+// (slot was set to -1 everywhere before).  A grid-stride loop over the
+// n_cols * N elements, i-major; a column outside [0, K) is skipped (no access
+// is made with it) and flagged in the error word.
+// ---------------------------------------------------------------------------
+__global__ void store_build_kernel(const uint16_t* __restrict__ W, int N, int K, const int32_t* __restrict__ cols,
+                                   int n_cols, int32_t* __restrict__ slot, uint16_t* __restrict__ Wst) {
+  const int64_t total = static_cast<int64_t>(n_cols) * N;
+  for (int64_t e = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; e < total;
+       e += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int i = static_cast<int>(e / N), n = static_cast<int>(e % N);
+    const int k = cols[i];
+    if (k < 0 || k >= K) {
+      if (n == 0) atomicOr(&g_error_word, kErrBadColumn);
+      continue;
+    }
+    if (n == 0) slot[k] = i;
+    Wst[e] = W[static_cast<int64_t>(n) * K + k];
   }
 }
 

@@ -9,6 +9,7 @@
 // [-127, 127], and q = 0 when s == 0.
 #pragma once
 #include <cuda_fp16.h>
+#include <cuda_fp8.h>
 #include "sm100.cuh"
 
 namespace llmint8 {
@@ -65,6 +66,43 @@ __device__ __forceinline__ uint2 quant8(const uint4 v, float s, float inv, uint3
     out[i >> 2] |= (static_cast<uint32_t>(qi) & 0xFFu) << ((i & 3) * 8);
   }
   return make_uint2(out[0], out[1]);
+}
+
+// ---------------------------------------------------------------------------
+// FP8 E4M3 codes ('量化压缩实战' (tqpw.cn) §3.6: 1 sign, 4 exponent, 3 mantissa
+// bits, largest finite 448): the same absmax recipe with 448 in place of 127,
+// s = amax / 448, code = e4m3(fl(x / s)), rounded to nearest even and
+// saturated to +-448 by the hardware conversion; s == 0 gives code 0.
+// ---------------------------------------------------------------------------
+template <bool FP8>
+__host__ __device__ constexpr float code_max() {
+  return FP8 ? 448.0f : 127.0f;
+}
+
+__device__ __forceinline__ uint32_t e4m3_code(float v, float s) {
+  if (s == 0.0f) return 0u;
+  return static_cast<uint32_t>(__nv_cvt_float_to_fp8(__fdiv_rn(v, s), __NV_SATFINITE, __NV_E4M3));
+}
+
+// Eight halves -> eight E4M3 codes (lanes set in `skip` get 0).
+__device__ __forceinline__ uint2 quant8_e4m3(const uint4 v, float s, uint32_t skip) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  uint32_t out[2] = {0u, 0u};
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const uint32_t c = ((skip >> i) & 1u) ? 0u : e4m3_code(half_bits_to_float(w[i >> 1] >> ((i & 1) * 16)), s);
+    out[i >> 2] |= c << ((i & 3) * 8);
+  }
+  return make_uint2(out[0], out[1]);
+}
+
+// Codes of either format; `inv` (= fl(1/s)) is used by the int8 codes only.
+template <bool FP8>
+__device__ __forceinline__ uint2 quant8_codes(const uint4 v, float s, float inv, uint32_t skip) {
+  if constexpr (FP8)
+    return quant8_e4m3(v, s, skip);
+  else
+    return quant8(v, s, inv, skip);
 }
 
 // max |x| over the lanes of eight halves whose bit is clear in `skip`.

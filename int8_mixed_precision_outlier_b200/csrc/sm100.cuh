@@ -25,6 +25,7 @@ enum : uint32_t {
   kErrTimeoutMma = 1u << 1,
   kErrTimeoutEpilogue = 1u << 2,
   kErrTimeoutSelftest = 1u << 3,
+  kErrBadColumn = 1u << 4,  // a column index outside [0, K) reached a kernel
 };
 
 // One word per device (this library is a single translation unit).
@@ -197,6 +198,13 @@ __device__ __forceinline__ void prefetch_l2(const void* p) {
   asm volatile("prefetch.global.L2 [%0];" ::"l"(reinterpret_cast<uint64_t>(p)) : "memory");
 }
 
+// Prefetch `bytes` (a multiple of 16) from a 16-byte aligned global address
+// into L2 with one bulk request; no data comes back to the SM.
+__device__ __forceinline__ void bulk_prefetch_l2(const void* p, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(p)), "r"(bytes)
+               : "memory");
+}
+
 // Prefetch one tensor-map box into L2 (x: a multiple of 16 bytes, as for loads).
 __device__ __forceinline__ void tma_prefetch_l2_2d(const CUtensorMap* map, int32_t x, int32_t y) {
   asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(
@@ -277,7 +285,23 @@ __host__ __device__ constexpr uint32_t idesc_f16_f32(int M, int N) {
          (static_cast<uint32_t>(M >> 4) << 24);
 }
 
+// kind::f8f6f4 with both operands E4M3 (type code 0) and an f32 accumulator:
+// the same field layout as idesc_f16_f32 (f16 is type code 0 of kind::f16).
+__host__ __device__ constexpr uint32_t idesc_e4m3_f32(int M, int N) {
+  return (1u << 4) | (0u << 7) | (0u << 10) | (static_cast<uint32_t>(N >> 3) << 17) |
+         (static_cast<uint32_t>(M >> 4) << 24);
+}
+
 // D[tmem] (+)= A[smem] * B[smem]^T, one instruction, issued by one thread.
+__device__ __forceinline__ void mma_f8(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                       uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
 __device__ __forceinline__ void mma_i8(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
                                        uint32_t idesc, uint32_t accumulate) {
   asm volatile(
@@ -347,6 +371,46 @@ __device__ __forceinline__ void mma_f16_pair(uint32_t d_tmem, uint64_t adesc, ui
       "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
+__device__ __forceinline__ void mma_f8_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                            uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// The 8-bit product of the two code formats: kind::i8 (signed int8, int32
+// accumulator) or kind::f8f6f4 (E4M3, f32 accumulator).
+template <bool FP8>
+__host__ __device__ constexpr uint32_t idesc_codes(int M, int N) {
+  return FP8 ? idesc_e4m3_f32(M, N) : idesc_i8_s32(M, N);
+}
+template <bool FP8>
+__device__ __forceinline__ void mma_codes(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+  if constexpr (FP8)
+    mma_f8(d, a, b, idesc, acc);
+  else
+    mma_i8(d, a, b, idesc, acc);
+}
+template <bool FP8>
+__device__ __forceinline__ void mma_codes_pair(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+  if constexpr (FP8)
+    mma_f8_pair(d, a, b, idesc, acc);
+  else
+    mma_i8_pair(d, a, b, idesc, acc);
+}
+// The accumulator of an 8-bit product as a float: int32 for int8 codes, the
+// f32 bits themselves for E4M3 codes.
+template <bool FP8>
+__device__ __forceinline__ float acc_value(uint32_t r) {
+  if constexpr (FP8)
+    return __uint_as_float(r);
+  else
+    return static_cast<float>(static_cast<int32_t>(r));
+}
+
 // Arrive once on `bar` (same shared-memory offset) in every CTA of `cta_mask`
 // when the issuing thread's earlier pair MMAs have completed.
 __device__ __forceinline__ void mma_commit_pair(uint64_t* bar, uint16_t cta_mask) {
@@ -477,6 +541,10 @@ __device__ __forceinline__ bool named_barrier_and(uint32_t id, uint32_t nthreads
       : "memory");
   return r != 0;
 }
+
+// |O| from device memory; a null pointer stands for no outlier columns (the
+// plain int8 product of llmint8_int8_gemm_i32).
+__device__ __forceinline__ int load_count(const int32_t* p) { return p ? *p : 0; }
 
 __device__ __forceinline__ uint32_t lane_id() { return threadIdx.x & 31u; }
 __device__ __forceinline__ uint32_t warp_id() { return threadIdx.x >> 5; }

@@ -162,10 +162,17 @@ def smoothquant_matmul(X, s, Wq, sw, intermediates: bool = False):
 
 # ------------------------------------------------------------------ FP8 E4M3
 
+_E4M3_TABLE = None
+
+
 def e4m3_to_float(codes: np.ndarray) -> np.ndarray:
-    f = _lib().onext_e4m3_to_float
-    c = np.asarray(codes, dtype=np.uint8)
-    return np.array([f(int(v)) for v in c.ravel()], np.float32).reshape(c.shape)
+    """Values of E4M3 codes (float32), looked up in the table of all 256 codes
+    that onext_e4m3_to_float decodes."""
+    global _E4M3_TABLE
+    if _E4M3_TABLE is None:
+        f = _lib().onext_e4m3_to_float
+        _E4M3_TABLE = np.array([f(v) for v in range(256)], np.float32)
+    return _E4M3_TABLE[np.asarray(codes, dtype=np.uint8)]
 
 
 def float_to_e4m3(x: np.ndarray) -> np.ndarray:

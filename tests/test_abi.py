@@ -111,7 +111,7 @@ def test_noalloc_limits_checked_before_any_device_call(lib):
     f = lib.llmint8_matmul_decode_noalloc
     assert f(A, 17, 64, A, A, A, 8, 6.0, A, None) == -1        # T > 16: not a decode shape
     assert f(A, 4, 16384 + 16, A, A, A, 8, 6.0, A, None) == -1  # K past the scratch limit
-    assert f(A, 4, 64, A, A, A, 65536 + 1, 6.0, A, None) == -1  # N past the limit
+    assert f(A, 4, 64, A, A, A, 1 << 31, 6.0, A, None) == -1      # N past int32
     assert f(A, 4, 72, A, A, A, 8, 6.0, A, None) == -1          # K % 16 != 0
     assert f(A, -1, 64, A, A, A, 8, 6.0, A, None) == -1
     assert f(None, 0, 64, A, A, A, 8, 6.0, A, None) == 0        # empty problems are no-ops
@@ -139,3 +139,77 @@ def test_product_code_never_touches_the_oracle():
                 assert not re.search(r"^\s*(from|import)\s+oracle", src, re.M), f
                 assert "llmint8_oracle" not in src, f
                 assert "liboracle" not in src, f
+
+
+def test_binding_shape_checks_run_before_any_launch():
+    """check_matmul_shapes (run by every matmul wrapper before its C call)
+    refuses any buffer whose shape disagrees with X [T, K] and Wq [N, K]: the
+    C side sees only pointers and would read or write past the end."""
+    import torch
+    T, N, K = 4, 8, 64
+    X = torch.zeros((T, K), dtype=torch.float16)
+    Wq = torch.zeros((N, K), dtype=torch.int8)
+    sw = torch.zeros(N, dtype=torch.float32)
+    W = torch.zeros((N, K), dtype=torch.float16)
+    Y = torch.zeros((T, N), dtype=torch.float16)
+    L.check_matmul_shapes(X, Wq, sw, W, Y)            # consistent: no error
+    L.check_matmul_shapes(X, Wq, sw, None, Y)         # W optional
+    bad = [dict(W=torch.zeros((N, K - 16), dtype=torch.float16)),
+           dict(W=torch.zeros((N + 1, K), dtype=torch.float16)),
+           dict(Wscale=torch.zeros(N - 1, dtype=torch.float32)),
+           dict(Wq=torch.zeros((N, K - 16), dtype=torch.int8)),
+           dict(Y=torch.zeros((T, N - 1), dtype=torch.float16)),
+           dict(Y=torch.zeros((T + 1, N), dtype=torch.float16)),
+           dict(acc_out=torch.zeros((T, N - 1), dtype=torch.int32)),
+           dict(xq_out=torch.zeros((T, K - 16), dtype=torch.int8)),
+           dict(sx_out=torch.zeros(T - 1, dtype=torch.float32)),
+           dict(idx_out=torch.zeros(K - 1, dtype=torch.int32))]
+    for b in bad:
+        args = dict(X=X, Wq=Wq, Wscale=sw, W=W, Y=Y)
+        args.update(b)
+        with pytest.raises(ValueError):
+            L.check_matmul_shapes(**args)
+
+
+def test_int8_gemm_i32_validation_before_any_device_call(lib):
+    A = _fake(0x10000)
+    f = lib.llmint8_int8_gemm_i32
+    assert f(A, A, 4, 8, 72, A, None) == -2               # K % 16 != 0
+    assert f(A, A, 4, 8, 8, A, None) == -1                # K < 16
+    assert f(A, A, 4, 8, 65536 + 16, A, None) == -1       # K past the limit
+    assert f(_fake(0x10008), A, 4, 8, 64, A, None) == -2  # misaligned Xq
+    assert f(A, A, 4, 8, 64, _fake(0x10002), None) == -2  # misaligned acc
+    assert f(None, A, 4, 8, 64, A, None) == -1
+    assert f(A, A, -1, 8, 64, A, None) == -1
+    assert f(None, None, 0, 8, 64, None, None) == 0       # empty problems are no-ops
+    assert f(A, A, 4, 0, 64, A, None) == 0
+
+
+def test_smoothquant_validation_before_any_device_call(lib):
+    A = _fake(0x10000)
+    big = 1 << 40
+    assert lib.llmint8_smooth_factors(A, A, 64, 1.5, A, None) == -1           # alpha outside [0, 1]
+    assert lib.llmint8_smooth_factors(A, A, 64, float("nan"), A, None) == -1
+    assert lib.llmint8_smooth_factors(A, A, 0, 0.5, A, None) == 0             # empty
+    assert lib.llmint8_column_absmax(A, 4, 72, A, 0, None) == -2              # K % 16
+    assert lib.llmint8_column_absmax(_fake(0x10008), 4, 64, A, 0, None) == -2
+    assert lib.llmint8_smoothquant_quantize_weight(A, 8, 64, _fake(0x10004), A, A, None) == -2  # s misaligned
+    assert lib.llmint8_smoothquant_workspace_bytes(4, 72) == 0
+    assert lib.llmint8_smoothquant_workspace_bytes(2048, 4096) >= 2048 * 4096 + 4 * 2048
+    f = lib.llmint8_smoothquant_matmul
+    assert f(A, 4, 64, A, A, A, 8, A, A, 16, None) == -4                      # workspace too small
+    assert f(A, 4, 64, None, A, A, 8, A, A, big, None) == -1                  # no factors
+    assert f(A, 4, 64, A, A, A, 0, A, A, big, None) == 0                      # empty
+    d = lib.llmint8_smoothquant_matmul_debug
+    assert d(A, 17, 64, A, A, A, 8, A, A, big, 1, None, None, None, None) == -1  # GEMV path, T > 16
+
+
+def test_prefetch_next_validation(lib):
+    A = _fake(0x10000)
+    big = 1 << 40
+    f = lib.llmint8_matmul_prefetch_next
+    assert f(A, 4, 64, A, A, A, 8, 6.0, A, A, big, A, -16, None) == -1      # negative size
+    assert f(A, 4, 64, A, A, A, 8, 6.0, A, A, big, None, 64, None) == -1    # bytes without a pointer
+    assert f(A, 4, 64, A, A, A, 8, 6.0, A, A, big, _fake(0x10008), 64, None) == -2  # misaligned
+    assert f(A, 4, 64, A, A, A, 8, 6.0, A, A, big, A, 24, None) == -2       # not a multiple of 16
+    assert f(A, 4, 64, A, A, A, 8, float("nan"), A, A, big, A, 64, None) == -1

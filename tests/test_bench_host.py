@@ -72,14 +72,15 @@ def test_shrink_sample_recounts_bytes_and_ops():
     sw = np.zeros(N, np.float32)
     W = np.zeros((N, K), np.float16)
     nbytes = N * K + 4 * N + 2 * N * n_out + 2 * T * K + 2 * T * N
-    calls, n = bench.shrink_sample([(X, Wq, sw, W, 6.0, nbytes, 2 * T * N * K)], 0.25)
-    X2, Wq2, sw2, W2, tau, b2, o2 = calls[0]
-    assert n == 250 and Wq2.shape == (250, K) and W2.shape == (250, K) and sw2.shape == (250,)
+    fn = object()
+    calls, n = bench.shrink_sample([(fn, (X, Wq, sw, W, 6.0), nbytes, 2 * T * N * K)], 0.25)
+    fn2, (X2, Wq2, sw2, W2, tau), b2, o2 = calls[0]
+    assert fn2 is fn and n == 250 and Wq2.shape == (250, K) and W2.shape == (250, K) and sw2.shape == (250,)
     assert b2 == n * K + 4 * n + 2 * n * n_out + 2 * T * K + 2 * T * n
     assert o2 == 2 * T * n * K
     # prefill samples carry no byte count; a tiny fraction keeps one row
-    calls, n = bench.shrink_sample([(X, Wq, sw, W, 6.0, 0, 2 * T * N * K)], 1e-9)
-    assert n == 1 and calls[0][5] == 0 and calls[0][6] == 2 * T * K
+    calls, n = bench.shrink_sample([(fn, (X, Wq, sw, W, 6.0), 0, 2 * T * N * K)], 1e-9)
+    assert n == 1 and calls[0][2] == 0 and calls[0][3] == 2 * T * K
 
 
 def test_reference_arm_prints_the_contract_line():

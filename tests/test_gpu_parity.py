@@ -2,10 +2,10 @@
 
 Integer stages (Wq, Wscale, outlier set, Xq, sx, int32 acc) must match bit for
 bit; Y must satisfy |Y_gpu - Y_oracle| <= 1e-3 max|Y_oracle| + 1 fp16 ulp.
-Small cases compare every element; the full-size workloads compare every
-integer stage in full (the int32 accumulator of every row by Freivalds'
-projection check against the oracle's codes) and Y / acc element by element
-on sampled rows, computed by the oracle one row at a time.
+Every case compares every element, the full-size workloads (7B prefill, 13B
+up-projection, 70B up-projection at thresholds 4, 6 and inf) included: there a
+projection check of the int32 accumulator runs first as a quick filter, then
+the oracle's full int8 product and fp part.
 """
 import numpy as np
 import pytest
@@ -248,17 +248,21 @@ def test_decode_7b_full(L, oracle):
     ok_status(L)
 
 
-def sampled_rows(T, seed):
-    rng = np.random.default_rng(seed)
-    rows = {0, T - 1, min(127, T - 1), min(128, T - 1)}
-    rows.update(rng.choice(T, size=min(T, 4), replace=False).tolist())
-    return np.array(sorted(rows))
+def oracle_outlier_part(oracle, X, W, idx_o):
+    """The oracle's fp part X[:, O] W[:, O]^T, computed on the gathered outlier
+    columns: yo[t, n] = sum_j X[t, O_j] W[n, O_j] with the same terms in the
+    same ascending order as on the full matrices (so the same binary64 sums),
+    but reading contiguous rows, which keeps the full-size cases in seconds."""
+    Xo = np.ascontiguousarray(X[:, idx_o])
+    Wo = np.ascontiguousarray(W[:, idx_o])
+    return oracle.outlier_gemm(Xo, Wo, np.arange(idx_o.size, dtype=np.int32))
 
 
-def run_sampled(L, oracle, X, W, taus, seed=0):
-    """Full-size check: every integer stage in full (acc of all rows by
-    random projections, exact in int64), Y and acc element by element on
-    sampled rows."""
+def run_full_size(L, oracle, X, W, taus, seed=0):
+    """Full-size check, every element: the integer stages (Wq, sw, the outlier
+    list, Xq, sx) bit for bit, the int32 accumulator of all T x N outputs bit
+    for bit against the oracle's int8 product (after a fast projection
+    pre-check of every row), and every element of Y within the tolerance."""
     T, K = X.shape
     N = W.shape[0]
     Wq_o, sw_o = oracle.quantize_weight(W)
@@ -268,7 +272,6 @@ def run_sampled(L, oracle, X, W, taus, seed=0):
     assert_equal(host(sw).view(np.uint32), sw_o.view(np.uint32), "Wscale")
     ws = L.alloc_workspace(T, N, K, "cuda")
     acc = torch.empty((T, N), dtype=torch.int32, device="cuda")
-    rows = sampled_rows(T, seed)
     proj = projected_weights(Wq_o, seed=seed)
     for tau in taus:
         flag = oracle.detect_outliers(X, tau)
@@ -281,32 +284,98 @@ def run_sampled(L, oracle, X, W, taus, seed=0):
         Y = L.llmint8_matmul_debug(Xd, Wq, sw, Wd, tau, workspace=ws, acc_out=acc)
         torch.cuda.synchronize()
         ok_status(L)
-        Xs = np.ascontiguousarray(X[rows])
-        acc_o = oracle.int8_gemm(np.ascontiguousarray(Xq_o[rows]), Wq_o)
-        yo_o = oracle.outlier_gemm(Xs, W, idx_o)
-        Y_o = oracle.dequant_combine(acc_o, sx_o[rows], sw_o, yo_o)
         acc_h = host(acc)
-        assert_acc_exact(acc_h, Xq_o, proj, f"acc all rows tau={tau}")
-        assert_equal(acc_h[rows], acc_o, f"acc rows tau={tau}")
-        assert_y_close(host(Y[rows]), Y_o, f"Y rows tau={tau}")
-        # a property at any size: Y is finite and the last row was written
-        assert torch.isfinite(Y).all()
-    return rows
+        assert_acc_exact(acc_h, Xq_o, proj, f"acc projections tau={tau}")
+        acc_o = oracle.int8_gemm(Xq_o, Wq_o)
+        assert_equal(acc_h, acc_o, f"acc every element tau={tau}")
+        yo_o = oracle_outlier_part(oracle, X, W, idx_o) if idx_o.size else None
+        Y_o = oracle.dequant_combine(acc_o, sx_o, sw_o, yo_o)
+        del acc_o, yo_o
+        assert_y_close(host(Y), Y_o, f"Y every element tau={tau}")
+        del Y_o
 
 
 def test_prefill_7b(L, oracle):
     w = synth.workload("7b_prefill")
-    run_sampled(L, oracle, w["X"], w["W"], w["thresholds"], seed=1)
+    run_full_size(L, oracle, w["X"], w["W"], w["thresholds"], seed=1)
 
 
 def test_upproj_13b(L, oracle):
     w = synth.workload("13b_up")
-    run_sampled(L, oracle, w["X"], w["W"], w["thresholds"], seed=2)
+    run_full_size(L, oracle, w["X"], w["W"], w["thresholds"], seed=2)
 
 
 def test_upproj_70b_threshold_sweep(L, oracle):
     w = synth.workload("70b_up")
-    run_sampled(L, oracle, w["X"], w["W"], w["thresholds"], seed=3)
+    run_full_size(L, oracle, w["X"], w["W"], w["thresholds"], seed=3)
+
+
+@pytest.mark.parametrize("tau", [6.0, 0.0, float("inf")])
+def test_pair_gemm_many_tiles_per_pair(L, oracle, tau):
+    """Every resident CTA pair of the persistent GEMM runs several tiles
+    (T 600 = 3 row tiles, N 20000: hundreds of tiles for at most 74 pairs), so
+    the hand-over between a pair's tiles (accumulator drain, weight-scale
+    reload, outlier accumulator reset) is checked element by element."""
+    X, W = synth.random_case(600, 1024, 20000, seed=600, n_dims=5, mag=(6.0, 50.0))
+    run_full(L, oracle, X, W, tau, 2)
+
+
+# --------------------------------------------------------------- int8 product alone
+
+def saturated_codes(rng, T, K):
+    """int8 codes over the full range, with rows of all +127, all -127, all
+    -128 and alternating signs."""
+    A = rng.integers(-128, 128, size=(T, K), dtype=np.int16).astype(np.int8)
+    for r, v in enumerate((127, -127, -128)):
+        if r < T:
+            A[r] = v
+    if T > 3:
+        A[3] = np.where(np.arange(K) % 2 == 0, 127, -128).astype(np.int8)
+    return A
+
+
+@pytest.mark.parametrize("T,N,K", [(1, 300, 16), (5, 1001, 1040), (16, 4096, 4096), (17, 513, 272),
+                                   (100, 300, 2048), (129, 777, 1024), (300, 1000, 4160),
+                                   (600, 20000, 512)])
+def test_int8_gemm_i32_bitexact(L, oracle, T, N, K):
+    """acc = Xq Wq^T on arbitrary int8 codes (-128 included, saturated rows,
+    adversarial signs), through each of the three kernels (GEMV T <= 16, one-CTA
+    GEMM T <= 128, CTA-pair GEMM), with ragged T, N and K tails."""
+    rng = np.random.default_rng(T * 1000 + N + K)
+    Xq = saturated_codes(rng, T, K)
+    Wq = saturated_codes(rng, N, K)
+    acc = L.llmint8_int8_gemm_i32(dev(Xq), dev(Wq))
+    torch.cuda.synchronize()
+    ok_status(L)
+    assert_equal(host(acc), oracle.int8_gemm(Xq, Wq), "acc")
+
+
+@pytest.mark.parametrize("T", [3, 200])
+def test_int8_gemm_i32_largest_k(L, oracle, T):
+    """K = 65536 with every code at its extreme: |acc| reaches 65536 * 128^2 =
+    2^30 (all -128 against all -128), the largest sum the entry allows."""
+    K, N = 65536, 40
+    rng = np.random.default_rng(T)
+    Xq = saturated_codes(rng, T, K)
+    Wq = saturated_codes(rng, N, K)
+    acc = L.llmint8_int8_gemm_i32(dev(Xq), dev(Wq))
+    torch.cuda.synchronize()
+    ok_status(L)
+    acc_o = oracle.int8_gemm(Xq, Wq)
+    assert acc_o[2, 2] == 2 ** 30
+    assert_equal(host(acc), acc_o, "acc")
+
+
+def test_int8_gemm_i32_matches_the_matmul_accumulator(L, oracle):
+    """The codes llmint8_matmul forms, multiplied by the standalone entry, give
+    the accumulator the matmul itself reports."""
+    X, W = synth.random_case(300, 1024, 640, seed=31, n_dims=4)
+    Wd = dev(W)
+    Wq, sw = L.llmint8_quantize_weight(Wd)
+    _, acc, Xq, _, _ = L.llmint8_matmul_intermediates(dev(X), Wq, sw, Wd, 6.0)
+    acc2 = L.llmint8_int8_gemm_i32(Xq, Wq)
+    torch.cuda.synchronize()
+    assert_equal(host(acc2), host(acc), "int8 product alone vs inside the matmul")
 
 
 # --------------------------------------------------------------- robustness
@@ -432,3 +501,56 @@ def test_profile_repeats_recompute_same_y(L, oracle, path):
     assert_equal(host(Y1), host(Y0), "profile repeats")
     Wq_o, sw_o = oracle.quantize_weight(W)
     assert_y_close(host(Y1), oracle.matmul(X, Wq_o, sw_o, W, 6.0), "Y")
+
+
+@pytest.mark.parametrize("path", [1, 2])
+def test_weight_rewritten_just_before_a_call_is_seen(L, oracle, path):
+    """The kernels request Wq before the kernel queued ahead of them is done
+    (programmatic dependent launch).  A weight quantised into the same Wq
+    buffer right before a call, on the same stream, must still be the one the
+    call reads: the weight kernel does not let its dependents start early."""
+    T = 16 if path == 1 else 300
+    N, K = 1500, 2048
+    X, W1 = synth.random_case(T, K, N, seed=70 + path, n_dims=4)
+    W2 = synth.make_weight(N, K, seed=80 + path, sigma=0.07)
+    W1d, W2d, Xd = dev(W1), dev(W2), dev(X)
+    Wq, sw = L.llmint8_quantize_weight(W1d)
+    ws = L.alloc_workspace(T, N, K, "cuda", path)
+    Y1 = L.llmint8_matmul_debug(Xd, Wq, sw, W1d, 6.0, workspace=ws, path=path)
+    L.llmint8_quantize_weight(W2d, Wq, sw)          # overwrite in place, same stream
+    Y2 = L.llmint8_matmul_debug(Xd, Wq, sw, W2d, 6.0, workspace=ws, path=path)
+    Wq.copy_(torch.zeros_like(Wq))                   # a torch kernel writes Wq, then a call
+    Y3 = L.llmint8_matmul_debug(Xd, Wq, sw, W2d, 6.0, workspace=ws, path=path)
+    torch.cuda.synchronize()
+    ok_status(L)
+    Wq1, sw1 = oracle.quantize_weight(W1)
+    Wq2, sw2 = oracle.quantize_weight(W2)
+    assert_y_close(host(Y1), oracle.matmul(X, Wq1, sw1, W1, 6.0), "first weight")
+    assert_y_close(host(Y2), oracle.matmul(X, Wq2, sw2, W2, 6.0), "rewritten weight")
+    assert_y_close(host(Y3), oracle.matmul(X, np.zeros_like(Wq2), sw2, W2, 6.0), "zeroed codes")
+
+
+@pytest.mark.parametrize("T", [1, 16, 200])
+def test_prefetch_next_gives_the_same_bytes(L, oracle, T):
+    """llmint8_matmul_prefetch_next only adds a request for the next layer's
+    weights into L2: Y is the bytes of llmint8_matmul, and the next call (on
+    the prefetched weights) is unaffected."""
+    N, K = 3000, 2048
+    X, W1 = synth.random_case(T, K, N, seed=90 + T, n_dims=4)
+    W2 = synth.make_weight(N, K, seed=91 + T)
+    W1d, W2d, Xd = dev(W1), dev(W2), dev(X)
+    Wq1, sw1 = L.llmint8_quantize_weight(W1d)
+    Wq2, sw2 = L.llmint8_quantize_weight(W2d)
+    ws = L.alloc_workspace(T, N, K, "cuda")
+    Ya = torch.empty((T, N), dtype=torch.float16, device="cuda")
+    Yb = torch.empty_like(Ya)
+    L.llmint8_matmul_prefetch_next(Xd, Wq1, sw1, W1d, 6.0, ws, Ya, Wq2)
+    Y2a = L.llmint8_matmul(Xd, Wq2, sw2, W2d, 6.0, workspace=ws)
+    L.llmint8_matmul(Xd, Wq1, sw1, W1d, 6.0, workspace=ws, Y=Yb)
+    Y2b = L.llmint8_matmul(Xd, Wq2, sw2, W2d, 6.0, workspace=ws)
+    torch.cuda.synchronize()
+    ok_status(L)
+    assert_equal(host(Ya).view(np.uint16), host(Yb).view(np.uint16), "with and without the request")
+    assert_equal(host(Y2a).view(np.uint16), host(Y2b).view(np.uint16), "the next call")
+    Wq_o, sw_o = oracle.quantize_weight(W1)
+    assert_y_close(host(Ya), oracle.matmul(X, Wq_o, sw_o, W1, 6.0), "Y")
