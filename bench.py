@@ -263,14 +263,11 @@ class Workload:
     (llmint8_matmul_stored with the workload's systematic outlier dims in a
     column store and no fp16 W)."""
 
-    def __init__(self, name: str, device, seed: int = 0, taus=None, variant: str = "llmint8",
-                 prefetch_next: bool = True):
+    def __init__(self, name: str, device, seed: int = 0, taus=None, variant: str = "llmint8"):
         import torch
         import int8_mixed_precision_outlier_b200 as L
         assert variant in VARIANTS, variant
         self.L, self.name, self.device, self.variant = L, name, device, variant
-        # decode: each call asks L2 for the next call's weight codes (the next layer)
-        self.prefetch_next = prefetch_next and name == "7b_decode" and variant == "llmint8"
         cfg = synth.WORKLOADS[name]
         self.K, self.N = cfg["K"], cfg["N"]
         self.calls = []
@@ -288,8 +285,6 @@ class Workload:
             for tau in taus:
                 shared = self._add(w, w["T"], tau, ws, shared=shared)
             self.unit, self.kind = "TOPS", "tensor"
-        for i, c in enumerate(self.calls):
-            c["next_Wq"] = self.calls[i + 1]["Wq"] if self.prefetch_next and i + 1 < len(self.calls) else None
         torch.cuda.synchronize()
         self.bytes_per_step = sum(c["bytes"] for c in self.calls)
         self.ops_per_step = sum(c["ops"] for c in self.calls)
@@ -358,9 +353,6 @@ class Workload:
         L = self.L
         Y = c["Y"] if Y is None else Y
         if self.variant == "llmint8":
-            if c.get("next_Wq") is not None:
-                return L.llmint8_matmul_prefetch_next(c["X"], c["Wq"], c["sw"], c["W"], c["tau"], c["ws"], Y,
-                                                      c["next_Wq"])
             return L.llmint8_matmul(c["X"], c["Wq"], c["sw"], c["W"], c["tau"], c["ws"], Y)
         if self.variant == "fp8":
             return L.llmint8_fp8_matmul(c["X"], c["Wq"], c["sw"], c["W"], c["tau"], c["ws"], Y)
@@ -466,8 +458,7 @@ def decode_roofline(wl: Workload, ms_per_step: float, cold_ms: float, cold_algo:
     return {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
             "frac": round(achieved / peak, 4), "traffic": traffic,
             "kernel": "decode_prep_kernel + gemv_kernel, one call as it runs in the step "
-                      f"({len(wl.calls)} calls per step; step bytes / step time"
-                      + ("; each call requests the next layer's weight codes into L2)" if wl.prefetch_next else ")"),
+                      f"({len(wl.calls)} calls per step; step bytes / step time)",
             "peak_source": f"{peaks['source']} hbm_gbs (copy, burst)",
             "frac_of_published": round(achieved / PUBLISHED["hbm_gbs"], 4),
             "algo_bytes_per_launch": int(wl.bytes_per_step / len(wl.calls)),
@@ -665,10 +656,8 @@ def workload_config(name: str) -> dict:
     return d
 
 
-# (workload, variant, threshold): the entries of "also" at N = 1; "llmint8-noprefetch" is the
-# decode step with plain llmint8_matmul calls (no request for the next layer's weights)
-ALSO = [("7b_decode", "llmint8-noprefetch", 6.0),
-        ("7b_prefill", "llmint8", 6.0), ("13b_up", "llmint8", 6.0), ("70b_up", "llmint8", 6.0),
+# (workload, variant, threshold): the entries of "also" at N = 1
+ALSO = [("7b_prefill", "llmint8", 6.0), ("13b_up", "llmint8", 6.0), ("70b_up", "llmint8", 6.0),
         ("70b_up", "llmint8", 4.0), ("70b_up", "llmint8", float("inf")),
         ("7b_prefill", "fp8", 6.0), ("13b_up", "fp8", 6.0), ("7b_prefill", "smoothquant", None),
         ("13b_up", "smoothquant", None), ("7b_prefill", "stored", 6.0), ("7b_decode", "fp8", 6.0),
@@ -681,15 +670,12 @@ ORACLE_ROWS = {"7b_prefill": 256, "13b_up": 128, "70b_up": 16}
 def also_entry(name, variant, tau, device, peaks, flush, steps, oracle_budget_s):
     import torch
     taus = None if tau is None else (tau,)
-    prefetch = not variant.endswith("-noprefetch")
-    variant = variant.replace("-noprefetch", "")
-    w2 = Workload(name, device, taus=taus, variant=variant, prefetch_next=prefetch)
+    w2 = Workload(name, device, taus=taus, variant=variant)
     w2.capture()
     ms, ck = time_steps(w2, steps, 3, 1, flush, run=w2.graph.replay)
     status = w2.L.llmint8_sync_status()
     c = w2.calls[0]
-    entry = {"workload": name, "variant": variant if prefetch or w2.unit != "GB/s" else variant + " (no next-layer prefetch)",
-             "value": round(w2.metric_value(ms * 1e-3, steps), 2),
+    entry = {"workload": name, "variant": variant, "value": round(w2.metric_value(ms * 1e-3, steps), 2),
              "unit": w2.unit, "ms_per_step": round(ms / steps, 4), "n_outliers": c["nO"],
              "threshold": tau, "clocks": ck, "device_status": w2.L.llmint8_status_string(status),
              "resident_weight_bytes": w2.resident_weight_bytes()}
@@ -763,8 +749,7 @@ def run_ours(args):
         del wl
         torch.cuda.empty_cache()
         line["also"] = [also_entry(name, variant, tau, device, peaks, flush, args.also_steps, args.also_cpu_budget_s)
-                        for name, variant, tau in ALSO if not (name == args.workload and variant == "llmint8")
-                        and not (name != "7b_decode" and variant.endswith("-noprefetch"))]
+                        for name, variant, tau in ALSO if not (name == args.workload and variant == "llmint8")]
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:

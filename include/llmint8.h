@@ -126,23 +126,6 @@ LLMINT8_API int llmint8_matmul(const void* X, int64_t T, int64_t K, const int8_t
                    size_t workspace_bytes, void* stream);
 
 /*
- * llmint8_matmul followed, inside the same kernels, by a request to bring
- * `next_bytes` bytes at `next` into L2: the int8 weight codes of the call that
- * will follow on this stream (the next layer).  No counterpart in the pages:
- * decode reads every weight once per token ('三、模型量化' Q15), so each call is
- * a stream of its weights, and HBM sits idle while one call ends and the next
- * one quantises its activations; the request keeps HBM busy through that gap.
- * Only the decode path (T <= 16) issues it, after its own weight copies; the
- * prefill path ignores it.  It is a hint: results are those of llmint8_matmul,
- * and the next call reads its weights as usual.  next: 16-byte aligned device
- * pointer, next_bytes a multiple of 16 (0 = none).
- */
-LLMINT8_API int llmint8_matmul_prefetch_next(const void* X, int64_t T, int64_t K, const int8_t* Wq,
-                                             const float* Wscale, const void* W, int64_t N, float threshold,
-                                             void* Y, void* workspace, size_t workspace_bytes, const void* next,
-                                             int64_t next_bytes, void* stream);
-
-/*
  * Inspection variant of llmint8_matmul used by the parity tests: `path` picks
  * the kernel path (LLMINT8_PATH_*), and each non-NULL output receives an
  * intermediate of that very call (all device buffers, written in full):

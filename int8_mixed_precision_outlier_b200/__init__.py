@@ -11,5 +11,5 @@ from .llmint8 import (  # noqa: F401
     llmint8_status_string, llmint8_sync_status, llmint8_version, llmint8_workspace_bytes,
     load_library, llmint8_column_absmax, llmint8_smooth_factors, llmint8_smoothquant_quantize_weight,
     llmint8_smoothquant_matmul, llmint8_fp8_quantize_weight, llmint8_fp8_matmul, llmint8_outlier_store_build,
-    llmint8_matmul_stored, llmint8_matmul_prefetch_next,
+    llmint8_matmul_stored,
 )

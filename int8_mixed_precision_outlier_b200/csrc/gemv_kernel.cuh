@@ -82,8 +82,6 @@ struct Params {
   const int32_t* n_out;
   uint16_t* Y;
   int32_t* acc_out;   // optional int32 [T][N] (FP8: the f32 accumulator's bits)
-  const uint8_t* pf_next;  // optional: bytes to request into L2 for the call that follows
-  int64_t pf_bytes;        // (a multiple of 16; CTA c takes the c-th equal share)
   uint64_t wait_ns;
 };
 
@@ -255,18 +253,6 @@ __global__ void __launch_bounds__(THREADS, 1)
         load_b(i, s);
         ++issued;
       }
-      // Every copy of this call is requested: ask L2 for this CTA's share of
-      // the weights of the call that follows (the next layer), so that HBM
-      // keeps streaming through this call's tail and the next call's prep.
-      if (p.pf_next) {
-        const int64_t per = ((p.pf_bytes + gridDim.x - 1) / gridDim.x + 15) / 16 * 16;
-        const int64_t beg = per * blockIdx.x;
-        const int64_t end = beg + per < p.pf_bytes ? beg + per : p.pf_bytes;
-        for (int64_t a = beg; a < end; a += 32768) {
-          const int64_t sz = end - a < 32768 ? end - a : 32768;
-          bulk_prefetch_l2(p.pf_next + a, static_cast<uint32_t>(sz));
-        }
-      }
       // Leave no copy in flight: wait for the last loads of every stage.
       for (int i = issued - STAGES < 0 ? 0 : issued - STAGES; i < issued; ++i)
         mbar_wait(&full[i % STAGES], (i / STAGES) & 1, p.wait_ns, kErrTimeoutProducer);
@@ -317,10 +303,16 @@ __global__ void __launch_bounds__(THREADS, 1)
     const int etid = threadIdx.x - 64;       // 0..127
     const int nO = load_count(p.n_out);
     const int T = p.T;
-    if (p.n_miss && blockIdx.x == 0 && etid == 0) {
+    if (p.n_miss && blockIdx.x == 0) {  // the misses, counted by the 128 epilogue threads
+      __shared__ int miss_s;
+      if (etid == 0) miss_s = 0;
+      named_barrier(1, 128);
       int miss = 0;
-      for (int j = 0; j < nO; ++j) miss += p.slot[p.idx[j]] < 0 ? 1 : 0;
-      *p.n_miss = miss;
+      for (int j = etid; j < nO; j += 128) miss += p.slot[p.idx[j]] < 0 ? 1 : 0;
+      miss = __reduce_add_sync(0xffffffffu, miss);
+      if (lane == 0) atomicAdd(&miss_s, miss);
+      named_barrier(1, 128);
+      if (etid == 0) *p.n_miss = miss_s;
     }
     float sxr[TMAX];
 #pragma unroll

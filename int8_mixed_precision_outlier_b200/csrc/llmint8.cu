@@ -354,8 +354,6 @@ struct MainOps {
   const uint16_t* Wst = nullptr;
   const int8_t* Wqr = nullptr;
   int32_t* n_miss = nullptr;
-  const uint8_t* pf_next = nullptr;  // decode: weights of the next call to request into L2
-  int64_t pf_bytes = 0;
 };
 
 // Encodes the main kernel's tensor maps (so that a failure launches nothing),
@@ -400,8 +398,6 @@ int run_main(int path, int t, int n, int k, const int8_t* Wq, const MainOps& m, 
     p.n_miss = m.n_miss;
     p.Y = m.Y;
     p.acc_out = m.acc;
-    p.pf_next = m.pf_next;
-    p.pf_bytes = m.pf_bytes;
     p.wait_ns = wait_ns;
     CUtensorMap tw, tx;
     const bool maps_ok =
@@ -495,7 +491,7 @@ int matmul_impl(const void* Xv, int64_t T, int64_t K, const int8_t* Wq, const fl
                 const void* Wv, int64_t N, float threshold, void* Yv, void* workspace,
                 size_t ws_bytes, int path, const Inspect& ins, void* stream,
                 cudaEvent_t ev_begin = nullptr, cudaEvent_t ev_end = nullptr, int repeat = 1,
-                const ColumnStore* store = nullptr, const void* pf_next = nullptr, int64_t pf_bytes = 0) {
+                const ColumnStore* store = nullptr) {
   Layout L;
   int rc = check_common(Xv, T, K, threshold, workspace, ws_bytes, path, &L, N);
   if (rc != LLMINT8_OK) return rc;
@@ -534,10 +530,6 @@ int matmul_impl(const void* Xv, int64_t T, int64_t K, const int8_t* Wq, const fl
     m.xo = reinterpret_cast<const uint16_t*>(ws + L.xo);
     m.wo = reinterpret_cast<const uint16_t*>(ws + L.wo);
     m.ldo = L.ldo;
-  }
-  if (pf_next && pf_bytes > 0) {
-    m.pf_next = static_cast<const uint8_t*>(pf_next);
-    m.pf_bytes = pf_bytes;
   }
   ColumnStore cs;
   if (store) {
@@ -790,15 +782,6 @@ int llmint8_matmul(const void* X, int64_t T, int64_t K, const int8_t* Wq, const 
                    size_t workspace_bytes, void* stream) {
   return matmul_impl<false>(X, T, K, Wq, Wscale, W, N, threshold, Y, workspace, workspace_bytes,
                             LLMINT8_PATH_AUTO, Inspect{}, stream);
-}
-
-int llmint8_matmul_prefetch_next(const void* X, int64_t T, int64_t K, const int8_t* Wq, const float* Wscale,
-                                 const void* W, int64_t N, float threshold, void* Y, void* workspace,
-                                 size_t workspace_bytes, const void* next, int64_t next_bytes, void* stream) {
-  if (next_bytes < 0 || (next_bytes > 0 && !next)) return LLMINT8_ERR_INVALID_ARG;
-  if (next_bytes > 0 && (!aligned16(next) || next_bytes % 16 != 0)) return LLMINT8_ERR_ALIGNMENT;
-  return matmul_impl<false>(X, T, K, Wq, Wscale, W, N, threshold, Y, workspace, workspace_bytes,
-                            LLMINT8_PATH_AUTO, Inspect{}, stream, nullptr, nullptr, 1, nullptr, next, next_bytes);
 }
 
 int llmint8_matmul_debug(const void* X, int64_t T, int64_t K, const int8_t* Wq, const float* Wscale,

@@ -197,7 +197,7 @@ __global__ void __launch_bounds__(kCompactThreads) compact_kernel(
 // ---------------------------------------------------------------------------
 constexpr int kQuantThreads = 128;
 constexpr int kWoRowsPerCta = 8;
-constexpr int kStoreRowsPerCta = 64;  // column-store gather: 64 rows x 64 columns per tile
+constexpr int kStoreRowsPerCta = 32;  // column-store gather: 32 rows x 64 columns per tile
 constexpr int kGatherIdxCap = 1024;  // outlier indices staged in shared memory per gather CTA
 
 __device__ __forceinline__ float block128_max(float v, float* red) {
@@ -209,11 +209,12 @@ __device__ __forceinline__ float block128_max(float v, float* red) {
 }
 
 // Outlier weights from a column store instead of the fp16 weight (W null,
-// slot / Wst set): gather CTAs take 64 rows of Wo each and walk the outlier
-// columns 64 at a time through a shared-memory tile, reading 64 consecutive
-// rows of a stored column (128 contiguous bytes) and writing 64 consecutive
-// columns of Wo.  A column missing from the store gets fp16(fl(sw[n] *
-// Wq[n,k])); CTA 0 counts those misses into *n_miss.
+// slot / Wst set): gather CTAs take 32 rows of Wo each and walk the outlier
+// columns 64 at a time through a shared-memory tile: the tile's columns and
+// store slots are staged first, then every thread has 16 independent loads in
+// flight, reading 32 consecutive rows of a stored column (64 contiguous bytes)
+// and writing 64 consecutive columns of Wo.  A column missing from the store
+// gets fp16(fl(sw[n] * Wq[n,k])); CTA 0 counts those misses into *n_miss.
 struct ColumnStore {
   const int32_t* slot = nullptr;   // [K]: row of Wst holding column k, or -1
   const uint16_t* Wst = nullptr;   // fp16 [n_store][N]
@@ -231,37 +232,60 @@ __global__ void __launch_bounds__(kQuantThreads) quant_gather_kernel(
   __shared__ int32_t si[kGatherIdxCap];
   __shared__ float red[4];
   __shared__ uint16_t tile[kStoreRowsPerCta][64 + 2];
+  __shared__ int32_t tk[64], tslot[64];
   // No early trigger: the GEMM that follows takes a whole SM's shared memory
   // per CTA, so it launches only as this kernel's CTAs complete.
   pdl_wait();
   const int nO = *n_out;
   const int opad = (nO + 63) & ~63;
   if (static_cast<int>(blockIdx.x) < gather_ctas && !W) {
-    if (blockIdx.x == 0 && threadIdx.x == 0 && cs.n_miss) {
+    if (blockIdx.x == 0 && cs.n_miss) {  // the misses, counted by the whole CTA
+      __shared__ int miss_s;
+      if (threadIdx.x == 0) miss_s = 0;
+      __syncthreads();
       int miss = 0;
-      for (int j = 0; j < nO; ++j) miss += cs.slot[idx[j]] < 0 ? 1 : 0;
-      *cs.n_miss = miss;
+      for (int j = threadIdx.x; j < nO; j += kQuantThreads) miss += cs.slot[idx[j]] < 0 ? 1 : 0;
+      miss = __reduce_add_sync(0xffffffffu, miss);
+      if ((threadIdx.x & 31) == 0) atomicAdd(&miss_s, miss);
+      __syncthreads();
+      if (threadIdx.x == 0) *cs.n_miss = miss_s;
     }
     const int n0 = static_cast<int>(blockIdx.x) * kStoreRowsPerCta;
     const int rows = min(kStoreRowsPerCta, N - n0);
+    constexpr int PER = kStoreRowsPerCta * 64 / kQuantThreads;  // 16 elements per thread
     for (int j0 = 0; j0 < opad; j0 += 64) {
-      for (int e = threadIdx.x; e < kStoreRowsPerCta * 64; e += kQuantThreads) {
-        const int jj = e / kStoreRowsPerCta, r = e % kStoreRowsPerCta, j = j0 + jj;
-        uint16_t v = 0;
-        if (j < nO && r < rows) {
-          const int k = idx[j], sl = cs.slot[k], n = n0 + r;
-          v = sl >= 0 ? __ldg(cs.Wst + static_cast<int64_t>(sl) * N + n)
-                      : __half_as_ushort(__float2half_rn(
-                            __fmul_rn(cs.sw[n], static_cast<float>(cs.Wq[static_cast<int64_t>(n) * K + k]))));
-        }
-        tile[r][jj] = v;
+      __syncthreads();  // the previous tile has been written out
+      if (threadIdx.x < 64) {
+        const int j = j0 + static_cast<int>(threadIdx.x);
+        const int k = j < nO ? idx[j] : 0;
+        tk[threadIdx.x] = k;
+        tslot[threadIdx.x] = j < nO ? cs.slot[k] : -2;  // -2: padding column, zeros
       }
       __syncthreads();
-      for (int e = threadIdx.x; e < kStoreRowsPerCta * 64; e += kQuantThreads) {
+      uint16_t v[PER];
+#pragma unroll
+      for (int u = 0; u < PER; ++u) {
+        const int e = static_cast<int>(threadIdx.x) + kQuantThreads * u;
+        const int jj = e / kStoreRowsPerCta, r = e % kStoreRowsPerCta, n = n0 + r;
+        const int sl = tslot[jj];
+        v[u] = 0;
+        if (r < rows && sl != -2)
+          v[u] = sl >= 0 ? __ldg(cs.Wst + static_cast<int64_t>(sl) * N + n)
+                         : __half_as_ushort(__float2half_rn(__fmul_rn(
+                               __ldg(cs.sw + n), static_cast<float>(cs.Wq[static_cast<int64_t>(n) * K + tk[jj]]))));
+      }
+#pragma unroll
+      for (int u = 0; u < PER; ++u) {
+        const int e = static_cast<int>(threadIdx.x) + kQuantThreads * u;
+        tile[e % kStoreRowsPerCta][e / kStoreRowsPerCta] = v[u];
+      }
+      __syncthreads();
+#pragma unroll
+      for (int u = 0; u < PER; ++u) {
+        const int e = static_cast<int>(threadIdx.x) + kQuantThreads * u;
         const int r = e / 64, jj = e % 64;
         if (r < rows) Wo[static_cast<int64_t>(n0 + r) * ldo + j0 + jj] = tile[r][jj];
       }
-      __syncthreads();
     }
     return;
   }

@@ -47,7 +47,6 @@ def _declare(lib):
         "llmint8_kernel_launches": (I, [I64, I64, I64, I]),
         "llmint8_matmul": (I, [P, I64, I64, P, P, P, I64, F, P, P, SZ, P]),
         "llmint8_matmul_debug": (I, [P, I64, I64, P, P, P, I64, F, P, P, SZ, I, P, P, P, P, P, P]),
-        "llmint8_matmul_prefetch_next": (I, [P, I64, I64, P, P, P, I64, F, P, P, SZ, P, I64, P]),
         "llmint8_matmul_profile": (I, [P, I64, I64, P, P, P, I64, F, P, P, SZ, I, I, P, P, P]),
         "llmint8_detect_quantize": (I, [P, I64, I64, F, P, P, P, P, P, SZ, I, P]),
         "llmint8_matmul_decode_noalloc": (I, [P, I64, I64, P, P, P, I64, F, P, P]),
@@ -200,27 +199,6 @@ def llmint8_matmul(X: torch.Tensor, Wq: torch.Tensor, Wscale: torch.Tensor, W: t
     """Y = X W^T by the LLM.int8() decomposition (fp16 [T,N])."""
     return llmint8_matmul_debug(X, Wq, Wscale, W, threshold, workspace, Y, PATH_AUTO, None,
                                 stream, _entry="llmint8_matmul")
-
-
-def llmint8_matmul_prefetch_next(X: torch.Tensor, Wq: torch.Tensor, Wscale: torch.Tensor, W: torch.Tensor,
-                                 threshold: float, workspace: torch.Tensor, Y: torch.Tensor,
-                                 next_weights: torch.Tensor | None, stream=None) -> torch.Tensor:
-    """llmint8_matmul, and (decode path) a request that brings `next_weights`
-    (the int8 codes of the next layer) into L2 while this call ends."""
-    for t, dt, nd, name in ((X, torch.float16, 2, "X"), (Wq, torch.int8, 2, "Wq"),
-                            (Wscale, torch.float32, 1, "Wscale"), (W, torch.float16, 2, "W"),
-                            (Y, torch.float16, 2, "Y"), (workspace, torch.uint8, 1, "workspace")):
-        _need(t, dt, nd, name)
-    check_matmul_shapes(X, Wq, Wscale, W, Y)
-    T, K = X.shape
-    N = Wq.shape[0]
-    nb = 0 if next_weights is None else next_weights.numel() * next_weights.element_size()
-    if next_weights is not None and (not next_weights.is_contiguous() or next_weights.device != X.device):
-        raise ValueError("next_weights must be a contiguous tensor on the device of X")
-    _check(load_library().llmint8_matmul_prefetch_next(
-        _ptr(X), T, K, _ptr(Wq), _ptr(Wscale), _ptr(W), N, float(threshold), _ptr(Y), _ptr(workspace),
-        workspace.numel(), _ptr(next_weights), nb - nb % 16, _stream(stream)), "llmint8_matmul_prefetch_next")
-    return Y
 
 
 def llmint8_matmul_decode_noalloc(X: torch.Tensor, Wq: torch.Tensor, Wscale: torch.Tensor,

@@ -202,14 +202,3 @@ def test_smoothquant_validation_before_any_device_call(lib):
     assert f(A, 4, 64, A, A, A, 0, A, A, big, None) == 0                      # empty
     d = lib.llmint8_smoothquant_matmul_debug
     assert d(A, 17, 64, A, A, A, 8, A, A, big, 1, None, None, None, None) == -1  # GEMV path, T > 16
-
-
-def test_prefetch_next_validation(lib):
-    A = _fake(0x10000)
-    big = 1 << 40
-    f = lib.llmint8_matmul_prefetch_next
-    assert f(A, 4, 64, A, A, A, 8, 6.0, A, A, big, A, -16, None) == -1      # negative size
-    assert f(A, 4, 64, A, A, A, 8, 6.0, A, A, big, None, 64, None) == -1    # bytes without a pointer
-    assert f(A, 4, 64, A, A, A, 8, 6.0, A, A, big, _fake(0x10008), 64, None) == -2  # misaligned
-    assert f(A, 4, 64, A, A, A, 8, 6.0, A, A, big, A, 24, None) == -2       # not a multiple of 16
-    assert f(A, 4, 64, A, A, A, 8, float("nan"), A, A, big, A, 64, None) == -1

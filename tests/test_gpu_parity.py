@@ -528,29 +528,3 @@ def test_weight_rewritten_just_before_a_call_is_seen(L, oracle, path):
     assert_y_close(host(Y1), oracle.matmul(X, Wq1, sw1, W1, 6.0), "first weight")
     assert_y_close(host(Y2), oracle.matmul(X, Wq2, sw2, W2, 6.0), "rewritten weight")
     assert_y_close(host(Y3), oracle.matmul(X, np.zeros_like(Wq2), sw2, W2, 6.0), "zeroed codes")
-
-
-@pytest.mark.parametrize("T", [1, 16, 200])
-def test_prefetch_next_gives_the_same_bytes(L, oracle, T):
-    """llmint8_matmul_prefetch_next only adds a request for the next layer's
-    weights into L2: Y is the bytes of llmint8_matmul, and the next call (on
-    the prefetched weights) is unaffected."""
-    N, K = 3000, 2048
-    X, W1 = synth.random_case(T, K, N, seed=90 + T, n_dims=4)
-    W2 = synth.make_weight(N, K, seed=91 + T)
-    W1d, W2d, Xd = dev(W1), dev(W2), dev(X)
-    Wq1, sw1 = L.llmint8_quantize_weight(W1d)
-    Wq2, sw2 = L.llmint8_quantize_weight(W2d)
-    ws = L.alloc_workspace(T, N, K, "cuda")
-    Ya = torch.empty((T, N), dtype=torch.float16, device="cuda")
-    Yb = torch.empty_like(Ya)
-    L.llmint8_matmul_prefetch_next(Xd, Wq1, sw1, W1d, 6.0, ws, Ya, Wq2)
-    Y2a = L.llmint8_matmul(Xd, Wq2, sw2, W2d, 6.0, workspace=ws)
-    L.llmint8_matmul(Xd, Wq1, sw1, W1d, 6.0, workspace=ws, Y=Yb)
-    Y2b = L.llmint8_matmul(Xd, Wq2, sw2, W2d, 6.0, workspace=ws)
-    torch.cuda.synchronize()
-    ok_status(L)
-    assert_equal(host(Ya).view(np.uint16), host(Yb).view(np.uint16), "with and without the request")
-    assert_equal(host(Y2a).view(np.uint16), host(Y2b).view(np.uint16), "the next call")
-    Wq_o, sw_o = oracle.quantize_weight(W1)
-    assert_y_close(host(Ya), oracle.matmul(X, Wq_o, sw_o, W1, 6.0), "Y")
