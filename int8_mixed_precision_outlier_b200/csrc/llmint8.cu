@@ -434,19 +434,24 @@ int run_main(int path, int t, int n, int k, const int8_t* Wq, const MainOps& m, 
   p.Y = m.Y;
   p.acc_out = m.acc;
   p.wait_ns = wait_ns;
-  // CTA pairs: the tile width whose tiles spread most evenly over the resident
-  // pairs, counting each tile's fixed cost as 32 more columns of work (a tie
-  // keeps the wider tile).
+  // CTA pairs: the tile width with the least estimated time.  A pair runs
+  // ceil(tiles / pairs) tiles one after the other; a tile costs one k-block
+  // step per 128 bytes of K plus the accumulator drain that the next tile's
+  // products wait for.  The step times are those measured on B200 for
+  // gemm_pair_kernel at bn = 256, 192, 128 (operands staged per step: 32, 28,
+  // 24 KiB per SM); a tie keeps the wider tile.
   p.bn = gemm::BN;
   if (pair) {
-    int64_t best = -1;
-    for (int bn : {256, 192, 128}) {
-      const int64_t tiles = static_cast<int64_t>(p.num_m) * ((n + bn - 1) / bn);
+    struct Choice { int bn; double step_us, drain_us; };
+    const Choice choices[] = {{256, 0.427, 1.4}, {192, 0.387, 1.05}, {128, 0.353, 0.7}};
+    double best = -1.0;
+    for (const Choice& c : choices) {
+      const int64_t tiles = static_cast<int64_t>(p.num_m) * ((n + c.bn - 1) / c.bn);
       const int64_t rounds = (tiles + max_pairs - 1) / max_pairs;
-      const int64_t cost = rounds * (bn + 32);
-      if (best < 0 || cost < best) {
+      const double cost = static_cast<double>(rounds) * (p.KB * c.step_us + c.drain_us);
+      if (best < 0.0 || cost < best * 0.999) {
         best = cost;
-        p.bn = bn;
+        p.bn = c.bn;
       }
     }
   }
@@ -458,13 +463,14 @@ int run_main(int path, int t, int n, int k, const int8_t* Wq, const MainOps& m, 
   std::memset(&ty, 0, sizeof(ty));
   if (p.y_tma && !encode_2d(&ty, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, m.Y, n, t, 2ull * n, gemm::P_YCOLS, gemm::BM))
     return LLMINT8_ERR_CUDA;
+  // rows of B per copy: this CTA's half of the pair's N = bn
+  const uint32_t b_rows = pair ? p.bn / 2 : gemm::BN;
   if (!encode_2d(&txq, CU_TENSOR_MAP_DATA_TYPE_UINT8, m.xq, k, t, k, gemm::BK, gemm::BM) ||
-      !encode_2d(&twq, CU_TENSOR_MAP_DATA_TYPE_UINT8, Wq, k, n, k, gemm::BK, pair ? p.bn / 2 : gemm::BN))
+      !encode_2d(&twq, CU_TENSOR_MAP_DATA_TYPE_UINT8, Wq, k, n, k, gemm::BK, b_rows))
     return LLMINT8_ERR_CUDA;
   if (m.xo) {
     if (!encode_2d(&txo, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, m.xo, m.ldo, t, 2ull * m.ldo, 64, gemm::BM) ||
-        !encode_2d(&two, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, m.wo, m.ldo, n, 2ull * m.ldo, 64,
-                   pair ? p.bn / 2 : gemm::BN))
+        !encode_2d(&two, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, m.wo, m.ldo, n, 2ull * m.ldo, 64, b_rows))
       return LLMINT8_ERR_CUDA;
   } else {
     // No outlier operands: |O| = 0, so the kernels never load through these.

@@ -190,8 +190,8 @@ __global__ void __launch_bounds__(kCompactThreads) compact_kernel(
 // [0, gather_ctas): 8 rows of W each -> Wo[n, 0:Opad) = W[n, idx] (zero past
 // |O|), listed first because their scattered loads take longest.  Blocks past
 // those: one row t of X each -> sx[t], Xq[t, :] and Xo[t, 0:Opad) = X[t, idx].
-// The row is read with 4 loads in flight per thread for its absmax, then
-// again (from L1, where this CTA just put it) for its codes.
+// The row is read with 4 loads in flight per thread for its absmax and, up to
+// K = 8192, kept in registers for its codes (longer rows are read again).
 // Opad = |O| rounded up to 64 (one 128-byte fp16 K block of the outlier GEMM).
 // FP8: E4M3 codes with sx = amax / 448 instead of int8 codes with amax / 127.
 // ---------------------------------------------------------------------------
@@ -325,9 +325,26 @@ __global__ void __launch_bounds__(kQuantThreads) quant_gather_kernel(
   const uint8_t* fb = reinterpret_cast<const uint8_t*>(flags);
   uint2* out = reinterpret_cast<uint2*>(Xq + t * K);
   const int nchunk = K >> 3;
-  constexpr int U = 4;  // loads in flight per thread
+  constexpr int U = 4;     // loads in flight per thread
+  constexpr int KEEP = 2;  // rounds whose values stay in registers for the second pass (K <= 8192)
+  constexpr int ROUND = kQuantThreads * U;
+  uint4 keep[KEEP][U];
   float m = 0.0f;
-  for (int c0 = threadIdx.x; c0 < nchunk; c0 += kQuantThreads * U) {
+  // pass 1: absmax over the regular columns; the first KEEP rounds of the row
+  // stay in registers, later rounds (K > 8192) are read again in pass 2
+#pragma unroll
+  for (int r = 0; r < KEEP; ++r) {
+    uint32_t f[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int c = static_cast<int>(threadIdx.x) + r * ROUND + kQuantThreads * u;
+      keep[r][u] = c < nchunk ? __ldg(row + c) : make_uint4(0u, 0u, 0u, 0u);
+      f[u] = c < nchunk ? __ldg(fb + c) : 0xFFu;
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) m = absmax8(keep[r][u], f[u], m);
+  }
+  for (int c0 = static_cast<int>(threadIdx.x) + KEEP * ROUND; c0 < nchunk; c0 += ROUND) {
     uint4 v[U];
     uint32_t f[U];
 #pragma unroll
@@ -342,8 +359,16 @@ __global__ void __launch_bounds__(kQuantThreads) quant_gather_kernel(
   const float s = __fdiv_rn(block128_max(m, red), code_max<FP8>());
   const float inv = scale_reciprocal(s);
   if (threadIdx.x == 0) sx[t] = s;
-  // second pass: the row was just read by this CTA and is still in L1
-  for (int c0 = threadIdx.x; c0 < nchunk; c0 += kQuantThreads * U) {
+  // pass 2: codes
+#pragma unroll
+  for (int r = 0; r < KEEP; ++r) {
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int c = static_cast<int>(threadIdx.x) + r * ROUND + kQuantThreads * u;
+      if (c < nchunk) out[c] = quant8_codes<FP8>(keep[r][u], s, inv, __ldg(fb + c));
+    }
+  }
+  for (int c0 = static_cast<int>(threadIdx.x) + KEEP * ROUND; c0 < nchunk; c0 += ROUND) {
     uint4 v[U];
     uint32_t f[U];
 #pragma unroll

@@ -320,6 +320,16 @@ def test_pair_gemm_many_tiles_per_pair(L, oracle, tau):
     run_full(L, oracle, X, W, tau, 2)
 
 
+@pytest.mark.parametrize("tau", [6.0, 0.0])
+def test_pair_gemm_ragged_edges(L, oracle, tau):
+    """Many pair tiles per CTA pair with a ragged last row tile (T 520), N not
+    a multiple of 8 (Y written with plain stores, a partial last tile) and K
+    not a multiple of 128; tau 0 makes every column an outlier, so the fp16
+    outlier products run over all of K; element by element."""
+    X, W = synth.random_case(520, 1040, 20001, seed=520, n_dims=5, mag=(6.0, 50.0))
+    run_full(L, oracle, X, W, tau, 2)
+
+
 # --------------------------------------------------------------- int8 product alone
 
 def saturated_codes(rng, T, K):
