@@ -95,8 +95,8 @@ LLMINT8_API size_t llmint8_workspace_bytes_path(int64_t T, int64_t N, int64_t K,
 
 /* How many kernels one llmint8_matmul call of this shape launches on `path`
  * (no counterpart in the pages; for launch accounting): 2 for the decode path
- * (prep + GEMV), 4 for the prefill path (detect, compact, quantize + gathers,
- * GEMM).  0 for shapes the path rejects or T == 0 / N == 0.  Host-only:
+ * (prep + GEMV), 3 for the prefill path (detection, quantisation with the
+ * compaction and gathers, GEMM).  0 for shapes the path rejects or T == 0 / N == 0.  Host-only:
  * touches no device. */
 LLMINT8_API int llmint8_kernel_launches(int64_t T, int64_t N, int64_t K, int path);
 

@@ -30,7 +30,6 @@ constexpr int kVersion = 100;  // 0.1.0
 constexpr int kMaxDevices = 64;
 constexpr int64_t kMaxK = 65536;         // decode prep keeps K/8 mask bytes in shared memory
 constexpr int64_t kMaxInt32Sum = 133143; // K * 127 * 127 < 2^31
-constexpr int kDetectTargetCtas = 592;   // 4 x 148 SMs
 
 std::atomic<uint64_t> g_wait_ns{2000000000ull};
 
@@ -178,8 +177,8 @@ size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 struct Layout {
   int path = 0;
-  int Kw = 0, R = 0, rows_per_chunk = 0, ldo = 0;
-  size_t part = 0, flags = 0, idx = 0, n_out = 0, sx = 0, xq = 0, xo = 0, wo = 0, total = 0;
+  int Kw = 0, rows_per_cta = 0, ldo = 0, nstrips = 0;
+  size_t rowmax = 0, flags = 0, idx = 0, n_out = 0, sx = 0, xq = 0, xo = 0, wo = 0, total = 0;
 };
 
 bool make_layout(int64_t T, int64_t N, int64_t K, int path, Layout* L) {
@@ -202,18 +201,11 @@ bool make_layout(int64_t T, int64_t N, int64_t K, int path, Layout* L) {
     L->xq = take(static_cast<size_t>(LLMINT8_GEMV_MAX_T) * K);
     // decode_workspace_bytes() states the same sum as a constant expression
   } else {
-    const int64_t strips = (K + kDetectCols - 1) / kDetectCols;
-    int64_t R = (kDetectTargetCtas + strips - 1) / strips;
-    const int64_t rmax = T > 0 ? (T + 3) / 4 : 1;
-    if (R > rmax) R = rmax;
-    if (R < 1) R = 1;
-    const int64_t rpc = T > 0 ? (T + R - 1) / R : 1;
-    R = T > 0 ? (T + rpc - 1) / rpc : 1;
-    L->R = static_cast<int>(R);
-    L->rows_per_chunk = static_cast<int>(rpc);
+    L->rows_per_cta = static_cast<int>(T > 0 ? (T + kDetectCluster - 1) / kDetectCluster : 1);
+    L->nstrips = static_cast<int>((K + kDetectCols - 1) / kDetectCols);
     L->ldo = static_cast<int>((K + 63) / 64 * 64);
-    L->part = take(sizeof(uint32_t) * static_cast<size_t>(R) * L->Kw);
     L->flags = take(sizeof(uint32_t) * L->Kw);
+    L->rowmax = take(sizeof(float) * static_cast<size_t>(T) * L->nstrips);
     L->idx = take(sizeof(int32_t) * K);
     L->n_out = take(sizeof(int32_t));
     L->sx = take(sizeof(float) * static_cast<size_t>(T));
@@ -281,8 +273,9 @@ struct Prep {
   int32_t* n_out;
 };
 
-// Activation stages.  Decode: one latency-oriented kernel.  Prefill: detect, compact,
-// quantize + gathers (the W gather only when W != nullptr).
+// Activation stages.  Decode: one latency-oriented kernel.  Prefill: detection (one
+// cluster of CTAs per column strip), then quantisation with the compaction and the
+// gathers (the W gather only when W != nullptr, the store gather with a column store).
 template <bool FP8>
 int launch_prep(const Layout& L, const uint16_t* X, int T, int K, const uint16_t* W, int N, float tau,
                 uint8_t* ws, const Prep& out, cudaStream_t st, const ColumnStore& cs = ColumnStore{}) {
@@ -295,20 +288,16 @@ int launch_prep(const Layout& L, const uint16_t* X, int T, int K, const uint16_t
                   out.sx, out.idx, out.n_out);
     return e == cudaSuccess ? LLMINT8_OK : LLMINT8_ERR_CUDA;
   }
-  uint32_t* part = reinterpret_cast<uint32_t*>(ws + L.part);
-  const int strips = (K + kDetectCols - 1) / kDetectCols;
-  e = launch(detect_partial_kernel, dim3(strips, L.R), dim3(kPrepThreads), 0, st, true, X, T, K, tau,
-             L.rows_per_chunk, part, L.Kw);
+  float* rowmax = reinterpret_cast<float*>(ws + L.rowmax);
+  e = launch_ex(detect_kernel, dim3(L.nstrips * kDetectCluster), dim3(kPrepThreads), 0, st, true, kDetectCluster, X,
+                T, K, tau, L.rows_per_cta, flags, L.Kw, rowmax, L.nstrips);
   if (e != cudaSuccess) return LLMINT8_ERR_CUDA;
-  e = launch(compact_kernel, dim3(1), dim3(kCompactThreads), 0, st, true,
-             static_cast<const uint32_t*>(part), L.R, L.Kw, flags, out.idx, out.n_out);
-  if (e != cudaSuccess) return LLMINT8_ERR_CUDA;
-  const int wblocks = W ? (N + kWoRowsPerCta - 1) / kWoRowsPerCta
-                      : cs.slot ? (N + kStoreRowsPerCta - 1) / kStoreRowsPerCta : 0;
-  e = launch(quant_gather_kernel<FP8>, dim3(wblocks + T), dim3(kQuantThreads), 0, st, true, X, T, K, W, N,
-             static_cast<const uint32_t*>(flags), static_cast<const int32_t*>(out.idx),
-             static_cast<const int32_t*>(out.n_out), out.xq, out.sx,
-             reinterpret_cast<uint16_t*>(ws + L.xo), reinterpret_cast<uint16_t*>(ws + L.wo), L.ldo, wblocks, cs);
+  const int gather_ctas = W ? (N + kWoRowsPerCta - 1) / kWoRowsPerCta
+                          : cs.slot ? (N + kStoreRowsPerCta - 1) / kStoreRowsPerCta : 0;
+  e = launch(quant_gather_kernel<FP8>, dim3(gather_ctas + T), dim3(kQuantThreads), 8 * static_cast<size_t>(L.Kw),
+             st, true, X, T, K, W, N, static_cast<const uint32_t*>(flags), L.Kw, static_cast<const float*>(rowmax),
+             L.nstrips, out.idx, out.n_out, out.xq, out.sx, reinterpret_cast<uint16_t*>(ws + L.xo),
+             reinterpret_cast<uint16_t*>(ws + L.wo), L.ldo, gather_ctas, cs);
   return e == cudaSuccess ? LLMINT8_OK : LLMINT8_ERR_CUDA;
 }
 
@@ -697,7 +686,7 @@ size_t llmint8_workspace_bytes_path(int64_t T, int64_t N, int64_t K, int path) {
 int llmint8_kernel_launches(int64_t T, int64_t N, int64_t K, int path) {
   Layout L;
   if (T <= 0 || N <= 0 || !make_layout(T, N, K, path, &L)) return 0;
-  return L.path == LLMINT8_PATH_GEMV ? 2 : 4;
+  return L.path == LLMINT8_PATH_GEMV ? 2 : 3;
 }
 
 size_t llmint8_workspace_bytes(int64_t T, int64_t N, int64_t K) {

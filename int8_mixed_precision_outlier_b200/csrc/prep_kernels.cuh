@@ -1,6 +1,6 @@
 // prep_kernels.cuh -- the HBM-bound stages of the LLM.int8() matmul:
 //   a0 weight quantisation (offline), a1 outlier detection, a4 compaction and
-//   gathers, a2+a3 per-row scale and int8 codes of X.
+//   gathers with a2+a3 per-row scale and int8 codes of X.
 //
 // Method: 'LLM quantization, part 2' (hncyxsy.com) §2.1 (vector-wise scales,
 // threshold 6.0 on activation magnitude, outlier columns leave the int8
@@ -85,127 +85,165 @@ __global__ void __launch_bounds__(kPrepThreads) quantize_weight_kernel(
 }
 
 // ---------------------------------------------------------------------------
-// a1 (prefill): partial outlier flags.  CTA (strip, chunk) covers 512 columns
-// x `rows_per_chunk` rows; thread (c = tid % 64, r = tid / 64) reads 16 B of
-// every 4th row.  Result: part[chunk][word] bitmasks, bit k%32 of word k/32.
+// a1 (prefill): the outlier flags, bit k%32 of word k/32 set iff some row has
+// |X[t,k]| >= tau, and the first half of a2: for every row t and 128-column
+// strip s, the maximum |X[t,k]| over the strip's regular columns,
+// rowmax[t * nstrips + s] (the row's absmax is the maximum of these).
+// A cluster of kDetectCluster CTAs owns a strip; CTA r scans rows
+// [r*rpc, (r+1)*rpc).  Thread (c = tid % 16, rr = tid / 16) reads the 16
+// bytes of chunk c in every 16th row, 8 rows in flight, and ORs 16-bit lane
+// masks (the bits are formed once at the end).  Every CTA sends its four
+// words to every CTA of the cluster (distributed shared memory), so after one
+// cluster barrier each holds the strip's final flags: the first CTA writes
+// them, and every CTA reads its rows again (from L1 / L2) for their maxima
+// over the unflagged columns, reduced over the 16 lanes of a row.
 // ---------------------------------------------------------------------------
-constexpr int kDetectCols = 512;
+constexpr int kDetectCols = 128;
+constexpr int kDetectCluster = 8;
 
-__global__ void __launch_bounds__(kPrepThreads) detect_partial_kernel(
-    const uint16_t* __restrict__ X, int T, int K, float tau, int rows_per_chunk,
-    uint32_t* __restrict__ part, int Kw) {
-  __shared__ uint32_t words[4][kDetectCols / 32];
-  const int c = threadIdx.x & 63, r = threadIdx.x >> 6;
-  if (threadIdx.x < 4 * (kDetectCols / 32)) (&words[0][0])[threadIdx.x] = 0u;
-  __syncthreads();
+__global__ void __launch_bounds__(kPrepThreads) detect_kernel(const uint16_t* __restrict__ X, int T, int K,
+                                                              float tau, int rpc, uint32_t* __restrict__ flags,
+                                                              int Kw, float* __restrict__ rowmax, int nstrips) {
+  constexpr int NW = kDetectCols / 32;  // flag words per strip
+  __shared__ uint32_t words[NW];
+  __shared__ uint32_t cw[kDetectCluster][NW];  // every CTA's words (each CTA holds a copy)
+  const int c = threadIdx.x & 15, rr = threadIdx.x >> 4;
+  const uint32_t rank = cluster_ctarank();
+  const int strip = blockIdx.x / kDetectCluster;
+  if (threadIdx.x < NW) words[threadIdx.x] = 0u;
   pdl_launch_dependents();
-  pdl_wait();  // X, and the workspace the previous call may still be reading
-  const int col0 = blockIdx.x * kDetectCols + c * 8;
-  const int t0 = blockIdx.y * rows_per_chunk;
-  const int t1 = min(T, t0 + rows_per_chunk);
-  uint32_t mask = 0;
-  if (col0 < K) {
-    const uint16_t* base = X + col0;
-    int t = t0 + r;
-    for (; t + 12 < t1; t += 16) {
-      const uint4 v0 = __ldg(reinterpret_cast<const uint4*>(base + (int64_t)t * K));
-      const uint4 v1 = __ldg(reinterpret_cast<const uint4*>(base + (int64_t)(t + 4) * K));
-      const uint4 v2 = __ldg(reinterpret_cast<const uint4*>(base + (int64_t)(t + 8) * K));
-      const uint4 v3 = __ldg(reinterpret_cast<const uint4*>(base + (int64_t)(t + 12) * K));
-      mask |= outlier_mask8(v0, tau) | outlier_mask8(v1, tau) | outlier_mask8(v2, tau) |
-              outlier_mask8(v3, tau);
-    }
-    for (; t < t1; t += 4)
-      mask |= outlier_mask8(__ldg(reinterpret_cast<const uint4*>(base + (int64_t)t * K)), tau);
-  }
-  if (mask) atomicOr(&words[r][c >> 2], mask << ((c & 3) * 8));
-  __syncthreads();
-  if (threadIdx.x < kDetectCols / 32) {
-    const int w = blockIdx.x * (kDetectCols / 32) + threadIdx.x;
-    if (w < Kw)
-      part[(int64_t)blockIdx.y * Kw + w] =
-          words[0][threadIdx.x] | words[1][threadIdx.x] | words[2][threadIdx.x] | words[3][threadIdx.x];
-  }
-}
-
-// ---------------------------------------------------------------------------
-// a4 (prefill): OR the partial flags, write the final bitmask and the
-// ascending outlier index list and its length.  One CTA of 1024 threads:
-// the R x Kw partial words are read with 8 loads in flight per thread and
-// OR-ed into shared words; then thread i owns words [i*wpt, (i+1)*wpt), so a
-// prefix sum of per-thread counts orders the indices.
-// ---------------------------------------------------------------------------
-constexpr int kCompactThreads = 1024;
-constexpr int kMaxKw = 65536 / 32;
-
-__global__ void __launch_bounds__(kCompactThreads) compact_kernel(
-    const uint32_t* __restrict__ part, int R, int Kw, uint32_t* __restrict__ flags,
-    int32_t* __restrict__ idx, int32_t* __restrict__ n_out) {
-  __shared__ uint32_t sw[kMaxKw];
-  __shared__ int scratch[33];
-  pdl_launch_dependents();
-  for (int w = threadIdx.x; w < Kw; w += kCompactThreads) sw[w] = 0u;
-  __syncthreads();
-  pdl_wait();
-  const int items = R * Kw;
+  cluster_sync();  // every CTA of the cluster runs before any remote store; words cleared
+  pdl_wait();      // X, and the workspace the previous call may still be reading
+  const int col0 = strip * kDetectCols + c * 8;
+  const int t0 = static_cast<int>(rank) * rpc;
+  const int t1 = min(T, t0 + rpc);
+  const bool live = col0 < K;
+  const uint16_t* base = X + col0;
   constexpr int U = 8;
-  for (int base = threadIdx.x; base < items; base += kCompactThreads * U) {
-    uint32_t v[U];
+  const __half2 tau2 = tau_half2(tau);
+  Mask8 acc = {{0u, 0u, 0u, 0u}};
+  if (live) {
+    int t = t0 + rr;
+    for (; t + 16 * (U - 1) < t1; t += 16 * U) {
+      uint4 v[U];
+#pragma unroll
+      for (int u = 0; u < U; ++u) v[u] = __ldg(reinterpret_cast<const uint4*>(base + static_cast<int64_t>(t + 16 * u) * K));
+#pragma unroll
+      for (int u = 0; u < U; ++u) outlier_mask8_or(v[u], tau2, acc);
+    }
+    for (; t < t1; t += 16) outlier_mask8_or(__ldg(reinterpret_cast<const uint4*>(base + static_cast<int64_t>(t) * K)), tau2, acc);
+  }
+  const uint32_t bits = mask_bits(acc);
+  if (bits) atomicOr(&words[c >> 2], bits << ((c & 3) * 8));
+  __syncthreads();
+  if (threadIdx.x < NW * kDetectCluster) {  // thread i: word i % NW to CTA i / NW
+    const uint32_t w = threadIdx.x % NW, dst = threadIdx.x / NW;
+    st_cluster_u32(map_shared_rank(&cw[rank][w], dst), words[w]);
+  }
+  cluster_sync();
+  uint32_t fw = 0;  // the strip's final word holding this thread's chunk
+#pragma unroll
+  for (int r = 0; r < kDetectCluster; ++r) fw |= cw[r][c >> 2];
+  if (rank == 0 && threadIdx.x < NW) {
+    uint32_t f = 0;
+#pragma unroll
+    for (int r = 0; r < kDetectCluster; ++r) f |= cw[r][threadIdx.x];
+    const int w = strip * NW + static_cast<int>(threadIdx.x);
+    if (w < Kw) flags[w] = f;
+  }
+  // the strip maxima of this CTA's rows over the regular columns
+  const uint32_t skip = live ? (fw >> ((c & 3) * 8)) & 0xFFu : 0xFFu;
+  const int rounds = (t1 - t0 + 15) / 16;  // uniform over the CTA (the shuffles need whole half-warps)
+  for (int i0 = 0; i0 < rounds; i0 += U) {
+    uint4 v[U];
 #pragma unroll
     for (int u = 0; u < U; ++u) {
-      const int e = base + u * kCompactThreads;
-      v[u] = e < items ? __ldg(part + e) : 0u;
+      const int t = t0 + rr + 16 * (i0 + u);
+      v[u] = (live && i0 + u < rounds && t < t1)
+                 ? __ldg(reinterpret_cast<const uint4*>(base + static_cast<int64_t>(t) * K))
+                 : make_uint4(0u, 0u, 0u, 0u);
     }
 #pragma unroll
-    for (int u = 0; u < U; ++u)
-      if (v[u]) atomicOr(&sw[(base + u * kCompactThreads) % Kw], v[u]);
-  }
-  __syncthreads();
-  const int wpt = (Kw + kCompactThreads - 1) / kCompactThreads;
-  const int w0 = threadIdx.x * wpt;
-  int count = 0;
-  for (int i = 0; i < wpt; ++i) {
-    const int w = w0 + i;
-    if (w >= Kw) break;
-    flags[w] = sw[w];
-    count += __popc(sw[w]);
-  }
-  int total;
-  int pos = block_exclusive_scan(count, scratch, &total);
-  for (int i = 0; i < wpt; ++i) {
-    const int w = w0 + i;
-    if (w >= Kw) break;
-    uint32_t f = sw[w];
-    while (f) {
-      const int b = __ffs(f) - 1;
-      idx[pos++] = w * 32 + b;
-      f &= f - 1;
+    for (int u = 0; u < U; ++u) {
+      float m = absmax8(v[u], skip, 0.0f);
+#pragma unroll
+      for (int o = 8; o >= 1; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+      const int t = t0 + rr + 16 * (i0 + u);
+      if (c == 0 && i0 + u < rounds && t < t1) rowmax[static_cast<int64_t>(t) * nstrips + strip] = m;
     }
   }
-  if (threadIdx.x == 0) *n_out = total;
 }
 
+constexpr int kMaxKw = 65536 / 32;
+
 // ---------------------------------------------------------------------------
-// a2 + a3 + a4 gathers (prefill), CTAs of 128 threads.  Blocks
-// [0, gather_ctas): 8 rows of W each -> Wo[n, 0:Opad) = W[n, idx] (zero past
-// |O|), listed first because their scattered loads take longest.  Blocks past
-// those: one row t of X each -> sx[t], Xq[t, :] and Xo[t, 0:Opad) = X[t, idx].
-// The row is read with 4 loads in flight per thread for its absmax and, up to
-// K = 8192, kept in registers for its codes (longer rows are read again).
+// a2 + a3 + a4 (prefill), CTAs of 128 threads.  Every CTA copies the Kw flag
+// words to shared memory and ranks them (exclusive prefix of the set bits per
+// word): outlier column j is the j-th set bit, |O| the total.  CTA 0 writes the
+// ascending index list and |O|.  Blocks [0, gather_ctas): 16 rows of W each ->
+// Wo[n, 0:Opad) = W[n, O] (zero past |O|), or 32 rows from a column store;
+// listed first because their scattered loads take longest.  Blocks past
+// those: one row t of X each, in one pass: sx[t] = (the maximum of the row's
+// strip maxima) / 127, Xq[t, :] and Xo[t, 0:Opad) = X[t, O], the outlier
+// values taken from the registers that hold the row.  The row's first loads
+// are issued before the flag words are ranked.
 // Opad = |O| rounded up to 64 (one 128-byte fp16 K block of the outlier GEMM).
 // FP8: E4M3 codes with sx = amax / 448 instead of int8 codes with amax / 127.
+// Dynamic shared memory: 8 * Kw bytes (flag words and their ranks).
 // ---------------------------------------------------------------------------
 constexpr int kQuantThreads = 128;
-constexpr int kWoRowsPerCta = 8;
+constexpr int kWoRowsPerCta = 16;
 constexpr int kStoreRowsPerCta = 32;  // column-store gather: 32 rows x 64 columns per tile
-constexpr int kGatherIdxCap = 1024;  // outlier indices staged in shared memory per gather CTA
+constexpr int kGatherIdxCap = 1024;  // outlier indices listed in shared memory at a time
 
-__device__ __forceinline__ float block128_max(float v, float* red) {
-  v = warp_max(v);
-  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
+// Outlier columns of rank j in [j0, j1) -> si[j - j0].  Thread i owns the
+// flag words [i * wpt, (i + 1) * wpt).
+__device__ __forceinline__ void list_outliers(const uint32_t* sf, const int32_t* wpre, int Kw, int j0, int j1,
+                                              int32_t* si) {
+  const int wpt = (Kw + kQuantThreads - 1) / kQuantThreads;
+  const int w0 = static_cast<int>(threadIdx.x) * wpt, w1 = min(Kw, w0 + wpt);
+  for (int w = w0; w < w1; ++w) {
+    int j = wpre[w];
+    if (j >= j1) break;
+    for (uint32_t f = sf[w]; f && j < j1; f &= f - 1, ++j)
+      if (j >= j0) si[j - j0] = w * 32 + __ffs(f) - 1;
+  }
+}
+
+// The flag words -> shared memory, ranked; returns |O|.  Thread i owns words
+// [i * wpt, (i + 1) * wpt).  Ends with a CTA barrier.
+__device__ __forceinline__ int rank_flags(const uint32_t* __restrict__ flags, int Kw, uint32_t* sf, int32_t* wpre,
+                                          int* scratch) {
+  const int wpt = (Kw + kQuantThreads - 1) / kQuantThreads;
+  const int w0 = static_cast<int>(threadIdx.x) * wpt, w1 = min(Kw, w0 + wpt);
+  int count = 0;
+  for (int w = w0; w < w1; ++w) {
+    const uint32_t f = __ldg(flags + w);
+    sf[w] = f;
+    count += __popc(f);
+  }
+  int nO;
+  int pos = block_exclusive_scan(count, scratch, &nO);
+  for (int w = w0; w < w1; ++w) {
+    wpre[w] = pos;
+    pos += __popc(sf[w]);
+  }
   __syncthreads();
-  const float r = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
-  return r;
+  return nO;
+}
+
+// Outlier columns of this chunk (bits of `fbits`, chunk c = columns 8c..8c+7)
+// -> Xo_row[rank]: the values are already in registers; ranks come from the
+// ranked flag words.
+__device__ __forceinline__ void emit_outliers(const uint4 v, int c, uint32_t fbits, const uint32_t* sf,
+                                              const int32_t* wpre, uint16_t* xo_row) {
+  const int w = c >> 2;
+  int j = wpre[w] + __popc(sf[w] & ((1u << ((c & 3) * 8)) - 1u));
+  for (uint32_t f = fbits; f; f &= f - 1) {
+    const int i = __ffs(f) - 1;
+    const uint32_t hw = i < 4 ? (i < 2 ? v.x : v.y) : (i < 6 ? v.z : v.w);
+    xo_row[j++] = static_cast<uint16_t>(hw >> ((i & 1) * 16));
+  }
 }
 
 // Outlier weights from a column store instead of the fp16 weight (W null,
@@ -224,167 +262,178 @@ struct ColumnStore {
 };
 
 template <bool FP8>
-__global__ void __launch_bounds__(kQuantThreads) quant_gather_kernel(
+__global__ void __launch_bounds__(kQuantThreads, 8) quant_gather_kernel(
     const uint16_t* __restrict__ X, int T, int K, const uint16_t* __restrict__ W, int N,
-    const uint32_t* __restrict__ flags, const int32_t* __restrict__ idx,
-    const int32_t* __restrict__ n_out, int8_t* __restrict__ Xq, float* __restrict__ sx,
+    const uint32_t* __restrict__ flags, int Kw, const float* __restrict__ rowmax, int nstrips,
+    int32_t* __restrict__ idx, int32_t* __restrict__ n_out, int8_t* __restrict__ Xq, float* __restrict__ sx,
     uint16_t* __restrict__ Xo, uint16_t* __restrict__ Wo, int ldo, int gather_ctas, const ColumnStore cs) {
+  extern __shared__ uint32_t sflags[];                          // [Kw] flag words, then [Kw] ranks
+  int32_t* wpre = reinterpret_cast<int32_t*>(sflags + Kw);
   __shared__ int32_t si[kGatherIdxCap];
-  __shared__ float red[4];
+  __shared__ int scratch[33];
   __shared__ uint16_t tile[kStoreRowsPerCta][64 + 2];
   __shared__ int32_t tk[64], tslot[64];
-  // No early trigger: the GEMM that follows takes a whole SM's shared memory
-  // per CTA, so it launches only as this kernel's CTAs complete.
+  // The GEMM that follows may launch once every CTA of this grid has started:
+  // its CTAs then take the SMs this grid's last CTAs leave and request their
+  // first weight tiles while those finish.
+  pdl_launch_dependents();
   pdl_wait();
-  const int nO = *n_out;
-  const int opad = (nO + 63) & ~63;
-  if (static_cast<int>(blockIdx.x) < gather_ctas && !W) {
-    if (blockIdx.x == 0 && cs.n_miss) {  // the misses, counted by the whole CTA
+  const int nchunk = K >> 3;
+  const bool xrow = static_cast<int>(blockIdx.x) >= gather_ctas;
+  // A row of X: its first round of loads goes out before the flags are ranked.
+  constexpr int U = 4;  // loads in flight per thread
+  constexpr int ROUND = kQuantThreads * U;
+  const int64_t t = static_cast<int64_t>(blockIdx.x) - gather_ctas;
+  const uint4* row = reinterpret_cast<const uint4*>(X + (xrow ? t : 0) * K);
+  uint4 v0[U];
+  float pm = 0.0f;
+  if (xrow) {
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int c = static_cast<int>(threadIdx.x) + kQuantThreads * u;
+      v0[u] = c < nchunk ? __ldg(row + c) : make_uint4(0u, 0u, 0u, 0u);
+    }
+    // every warp reduces the row's strip maxima itself (no CTA barrier)
+    for (int i = static_cast<int>(threadIdx.x & 31); i < nstrips; i += 32) pm = fmaxf(pm, __ldg(rowmax + t * nstrips + i));
+  }
+  const int nO = rank_flags(flags, Kw, sflags, wpre, scratch);
+  if (blockIdx.x == 0) {  // the index list and |O|, for the caller and the next kernels
+    const int wpt = (Kw + kQuantThreads - 1) / kQuantThreads;
+    const int w0 = static_cast<int>(threadIdx.x) * wpt, w1 = min(Kw, w0 + wpt);
+    for (int w = w0; w < w1; ++w) {
+      int j = wpre[w];
+      for (uint32_t f = sflags[w]; f; f &= f - 1) idx[j++] = w * 32 + __ffs(f) - 1;
+    }
+    if (threadIdx.x == 0) *n_out = nO;
+    if (cs.n_miss) {  // outlier columns the column store does not hold
       __shared__ int miss_s;
       if (threadIdx.x == 0) miss_s = 0;
       __syncthreads();
       int miss = 0;
-      for (int j = threadIdx.x; j < nO; j += kQuantThreads) miss += cs.slot[idx[j]] < 0 ? 1 : 0;
+      for (int w = threadIdx.x; w < Kw; w += kQuantThreads)
+        for (uint32_t f = sflags[w]; f; f &= f - 1) miss += cs.slot[w * 32 + __ffs(f) - 1] < 0 ? 1 : 0;
       miss = __reduce_add_sync(0xffffffffu, miss);
       if ((threadIdx.x & 31) == 0) atomicAdd(&miss_s, miss);
       __syncthreads();
       if (threadIdx.x == 0) *cs.n_miss = miss_s;
     }
+  }
+  const int opad = (nO + 63) & ~63;
+  if (!xrow && !W) {
+    // ---------------------------------------------------- column-store gather
     const int n0 = static_cast<int>(blockIdx.x) * kStoreRowsPerCta;
     const int rows = min(kStoreRowsPerCta, N - n0);
     constexpr int PER = kStoreRowsPerCta * 64 / kQuantThreads;  // 16 elements per thread
-    for (int j0 = 0; j0 < opad; j0 += 64) {
-      __syncthreads();  // the previous tile has been written out
-      if (threadIdx.x < 64) {
-        const int j = j0 + static_cast<int>(threadIdx.x);
-        const int k = j < nO ? idx[j] : 0;
-        tk[threadIdx.x] = k;
-        tslot[threadIdx.x] = j < nO ? cs.slot[k] : -2;  // -2: padding column, zeros
-      }
-      __syncthreads();
-      uint16_t v[PER];
+    for (int win = 0; win < opad; win += kGatherIdxCap) {
+      __syncthreads();  // the previous window's indices have been read
+      list_outliers(sflags, wpre, Kw, win, min(nO, win + kGatherIdxCap), si);
+      for (int j0 = win; j0 < min(opad, win + kGatherIdxCap); j0 += 64) {
+        __syncthreads();  // si is complete; the previous tile has been written out
+        if (threadIdx.x < 64) {
+          const int j = j0 + static_cast<int>(threadIdx.x);
+          const int k = j < nO ? si[j - win] : 0;
+          tk[threadIdx.x] = k;
+          tslot[threadIdx.x] = j < nO ? cs.slot[k] : -2;  // -2: padding column, zeros
+        }
+        __syncthreads();
+        uint16_t v[PER];
 #pragma unroll
-      for (int u = 0; u < PER; ++u) {
-        const int e = static_cast<int>(threadIdx.x) + kQuantThreads * u;
-        const int jj = e / kStoreRowsPerCta, r = e % kStoreRowsPerCta, n = n0 + r;
-        const int sl = tslot[jj];
-        v[u] = 0;
-        if (r < rows && sl != -2)
-          v[u] = sl >= 0 ? __ldg(cs.Wst + static_cast<int64_t>(sl) * N + n)
-                         : __half_as_ushort(__float2half_rn(__fmul_rn(
-                               __ldg(cs.sw + n), static_cast<float>(cs.Wq[static_cast<int64_t>(n) * K + tk[jj]]))));
-      }
+        for (int u = 0; u < PER; ++u) {
+          const int e = static_cast<int>(threadIdx.x) + kQuantThreads * u;
+          const int jj = e / kStoreRowsPerCta, r = e % kStoreRowsPerCta, n = n0 + r;
+          const int sl = tslot[jj];
+          v[u] = 0;
+          if (r < rows && sl != -2)
+            v[u] = sl >= 0 ? __ldg(cs.Wst + static_cast<int64_t>(sl) * N + n)
+                           : __half_as_ushort(__float2half_rn(__fmul_rn(
+                                 __ldg(cs.sw + n), static_cast<float>(cs.Wq[static_cast<int64_t>(n) * K + tk[jj]]))));
+        }
 #pragma unroll
-      for (int u = 0; u < PER; ++u) {
-        const int e = static_cast<int>(threadIdx.x) + kQuantThreads * u;
-        tile[e % kStoreRowsPerCta][e / kStoreRowsPerCta] = v[u];
-      }
-      __syncthreads();
+        for (int u = 0; u < PER; ++u) {
+          const int e = static_cast<int>(threadIdx.x) + kQuantThreads * u;
+          tile[e % kStoreRowsPerCta][e / kStoreRowsPerCta] = v[u];
+        }
+        __syncthreads();
 #pragma unroll
-      for (int u = 0; u < PER; ++u) {
-        const int e = static_cast<int>(threadIdx.x) + kQuantThreads * u;
-        const int r = e / 64, jj = e % 64;
-        if (r < rows) Wo[static_cast<int64_t>(n0 + r) * ldo + j0 + jj] = tile[r][jj];
+        for (int u = 0; u < PER; ++u) {
+          const int e = static_cast<int>(threadIdx.x) + kQuantThreads * u;
+          const int r = e / 64, jj = e % 64;
+          if (r < rows) Wo[static_cast<int64_t>(n0 + r) * ldo + j0 + jj] = tile[r][jj];
+        }
       }
     }
     return;
   }
-  if (static_cast<int>(blockIdx.x) < gather_ctas) {
-    const int nstage = nO < kGatherIdxCap ? nO : kGatherIdxCap;
-    for (int j = threadIdx.x; j < nstage; j += blockDim.x) si[j] = idx[j];
-    __syncthreads();
+  if (!xrow) {
+    // ---------------------------------------------------- fp16 weight gather
     const int64_t n0 = static_cast<int64_t>(blockIdx.x) * kWoRowsPerCta;
     const int64_t left = static_cast<int64_t>(N) - n0;
     const int rows = left < kWoRowsPerCta ? static_cast<int>(left) : kWoRowsPerCta;
-    const int total = rows * opad;
-    constexpr int U = 8;
-    for (int base = threadIdx.x; base < total; base += U * blockDim.x) {
-      uint16_t v[U];
+    for (int win = 0; win < opad; win += kGatherIdxCap) {
+      __syncthreads();  // the previous window's indices have been read
+      list_outliers(sflags, wpre, Kw, win, min(nO, win + kGatherIdxCap), si);
+      __syncthreads();
+      const int width = min(opad - win, kGatherIdxCap);
+      const int total = rows * width;
+      constexpr int UG = 8;
+      for (int base = threadIdx.x; base < total; base += UG * kQuantThreads) {
+        uint16_t v[UG];
 #pragma unroll
-      for (int u = 0; u < U; ++u) {
-        const int e = base + u * blockDim.x;
-        v[u] = 0;
-        if (e < total) {
-          const int rr = e / opad, j = e - rr * opad;
-          if (j < nO) v[u] = __ldg(W + (n0 + rr) * K + (j < kGatherIdxCap ? si[j] : idx[j]));
+        for (int u = 0; u < UG; ++u) {
+          const int e = base + u * kQuantThreads;
+          v[u] = 0;
+          if (e < total) {
+            const int rr = e / width, jj = e - rr * width;
+            if (win + jj < nO) v[u] = __ldg(W + (n0 + rr) * K + si[jj]);
+          }
         }
-      }
 #pragma unroll
-      for (int u = 0; u < U; ++u) {
-        const int e = base + u * blockDim.x;
-        if (e < total) {
-          const int rr = e / opad, j = e - rr * opad;
-          Wo[(n0 + rr) * ldo + j] = v[u];
+        for (int u = 0; u < UG; ++u) {
+          const int e = base + u * kQuantThreads;
+          if (e < total) {
+            const int rr = e / width, jj = e - rr * width;
+            Wo[(n0 + rr) * ldo + win + jj] = v[u];
+          }
         }
       }
     }
     return;
   }
-  const int64_t t = blockIdx.x - gather_ctas;
-  const uint4* row = reinterpret_cast<const uint4*>(X + t * K);
-  const uint8_t* fb = reinterpret_cast<const uint8_t*>(flags);
-  uint2* out = reinterpret_cast<uint2*>(Xq + t * K);
-  const int nchunk = K >> 3;
-  constexpr int U = 4;     // loads in flight per thread
-  constexpr int KEEP = 2;  // rounds whose values stay in registers for the second pass (K <= 8192)
-  constexpr int ROUND = kQuantThreads * U;
-  uint4 keep[KEEP][U];
-  float m = 0.0f;
-  // pass 1: absmax over the regular columns; the first KEEP rounds of the row
-  // stay in registers, later rounds (K > 8192) are read again in pass 2
-#pragma unroll
-  for (int r = 0; r < KEEP; ++r) {
-    uint32_t f[U];
-#pragma unroll
-    for (int u = 0; u < U; ++u) {
-      const int c = static_cast<int>(threadIdx.x) + r * ROUND + kQuantThreads * u;
-      keep[r][u] = c < nchunk ? __ldg(row + c) : make_uint4(0u, 0u, 0u, 0u);
-      f[u] = c < nchunk ? __ldg(fb + c) : 0xFFu;
-    }
-#pragma unroll
-    for (int u = 0; u < U; ++u) m = absmax8(keep[r][u], f[u], m);
-  }
-  for (int c0 = static_cast<int>(threadIdx.x) + KEEP * ROUND; c0 < nchunk; c0 += ROUND) {
-    uint4 v[U];
-    uint32_t f[U];
-#pragma unroll
-    for (int u = 0; u < U; ++u) {
-      const int c = c0 + kQuantThreads * u;
-      v[u] = c < nchunk ? __ldg(row + c) : make_uint4(0u, 0u, 0u, 0u);
-      f[u] = c < nchunk ? __ldg(fb + c) : 0xFFu;
-    }
-#pragma unroll
-    for (int u = 0; u < U; ++u) m = absmax8(v[u], f[u], m);
-  }
-  const float s = __fdiv_rn(block128_max(m, red), code_max<FP8>());
+  // ------------------------------------------------------ one row of X, one pass
+  pm = warp_max(pm);
+  const float s = __fdiv_rn(pm, code_max<FP8>());
   const float inv = scale_reciprocal(s);
   if (threadIdx.x == 0) sx[t] = s;
-  // pass 2: codes
+  const uint8_t* fb = reinterpret_cast<const uint8_t*>(sflags);  // byte c: the flags of chunk c
+  uint2* out = reinterpret_cast<uint2*>(Xq + t * K);
+  uint16_t* xo_row = Xo + t * ldo;
 #pragma unroll
-  for (int r = 0; r < KEEP; ++r) {
-#pragma unroll
-    for (int u = 0; u < U; ++u) {
-      const int c = static_cast<int>(threadIdx.x) + r * ROUND + kQuantThreads * u;
-      if (c < nchunk) out[c] = quant8_codes<FP8>(keep[r][u], s, inv, __ldg(fb + c));
+  for (int u = 0; u < U; ++u) {
+    const int c = static_cast<int>(threadIdx.x) + kQuantThreads * u;
+    if (c < nchunk) {
+      const uint32_t f = fb[c];
+      out[c] = quant8_codes<FP8>(v0[u], s, inv, f);
+      if (f) emit_outliers(v0[u], c, f, sflags, wpre, xo_row);
     }
   }
-  for (int c0 = static_cast<int>(threadIdx.x) + KEEP * ROUND; c0 < nchunk; c0 += ROUND) {
+  for (int c0 = static_cast<int>(threadIdx.x) + ROUND; c0 < nchunk; c0 += ROUND) {
     uint4 v[U];
-    uint32_t f[U];
 #pragma unroll
     for (int u = 0; u < U; ++u) {
       const int c = c0 + kQuantThreads * u;
       v[u] = c < nchunk ? __ldg(row + c) : make_uint4(0u, 0u, 0u, 0u);
-      f[u] = c < nchunk ? __ldg(fb + c) : 0xFFu;
     }
 #pragma unroll
     for (int u = 0; u < U; ++u) {
       const int c = c0 + kQuantThreads * u;
-      if (c < nchunk) out[c] = quant8_codes<FP8>(v[u], s, inv, f[u]);
+      if (c < nchunk) {
+        const uint32_t f = fb[c];
+        out[c] = quant8_codes<FP8>(v[u], s, inv, f);
+        if (f) emit_outliers(v[u], c, f, sflags, wpre, xo_row);
+      }
     }
   }
-  for (int j = threadIdx.x; j < opad; j += kQuantThreads)
-    Xo[t * ldo + j] = j < nO ? X[t * K + idx[j]] : uint16_t(0);
+  for (int j = nO + static_cast<int>(threadIdx.x); j < opad; j += kQuantThreads) xo_row[j] = uint16_t(0);
 }
 
 // ---------------------------------------------------------------------------
@@ -438,6 +487,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 4) decode_prep_kernel(
   // any later write of X), so it is safe however X is produced.
   for (int e = tid; e < items; e += kDecodeThreads)
     if (t < T && (e / TMAX) % 8 == 0) prefetch_l2(xrow + e / TMAX);
+  const __half2 tau2 = tau_half2(tau);
   cluster_sync();  // every CTA of the cluster has started before any remote access
   pdl_wait();
 
@@ -456,7 +506,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 4) decode_prep_kernel(
 #pragma unroll
     for (int u = 0; u < kDecodeInFlight; ++u) {
       const int e = base + u * kDecodeThreads;
-      uint32_t mask = outlier_mask8(v[u], tau) & (t < T ? 0xFFu : 0u);
+      uint32_t mask = outlier_mask8(v[u], tau2) & (t < T ? 0xFFu : 0u);
 #pragma unroll
       for (int o = 1; o < TMAX; o <<= 1) mask |= __shfl_xor_sync(0xffffffffu, mask, o);
       if (e < items && t == 0) fm[e / TMAX] = static_cast<uint8_t>(mask);

@@ -24,48 +24,79 @@ __device__ __forceinline__ int8_t quant_code(float x, float s) {
 }
 
 // The same code without a division in the common case.  With inv = fl(1/s)
-// (correctly rounded) and a = fl(x * inv):
-//   |a - x/s| <= |x/s| (2^-24 + 2^-24 + 2^-48) <= 2^-16,  since |x/s| <= 127 (1 + 2^-24);
+// (correctly rounded) and e = x * inv (the exact product):
+//   |e - x/s| <= |x/s| 2^-24 < 2^-17,  since |x/s| <= 127 (1 + 2^-23);
 //   |fl(x/s) - x/s| <= 2^-18 (half an ulp below 128).
-// So when a lies farther than 2^-12 from every half-integer k + 1/2, i.e. when
-// |a - rint(a)| < 1/2 - 2^-12, the values a, x/s and fl(x/s) all sit strictly
-// between the same two half-integers and round to the same integer, rint(a).
-// Only inside that band (about one element in 2000) is fl(x/s) formed by the
-// IEEE division.  A zero scale has inv = 0, so a = 0 and the code is 0.
+// So when e lies farther than 2^-16 from every half-integer k + 1/2, the
+// values e, x/s and fl(x/s) all sit strictly between the same two
+// half-integers and round to the same integer, rint(e).  Three fused or exact
+// steps give rint(e) and the distance to it (M = 1.5 * 2^23):
+//   t = fl(e + M)       one rounding to an integer: M + rint_even(e) for
+//                       |e| < 2^22; the low byte of t's bits is that integer
+//                       as a two's-complement byte (t - 2^23 = 2^22 + q);
+//   r = t - M           exact;
+//   d = fl(e - r)       the product stays exact inside the fused multiply-add,
+//                       so d is e - r rounded once (|error| <= 2^-25).
+// An element with |d| < 1/2 - 2^-12 is at least 2^-12 - 2^-25 > 2^-16 away
+// from every half-integer and takes the code of t.  The others (about one in
+// 2000, and NaN) get the IEEE division.  A regular element satisfies |x| <=
+// amax, hence |e| <= 127 (1 + 2^-23) and |rint(e)| <= 127: no clamp is needed
+// on the fast path.  A zero scale has inv = 0, so t = M and the code is 0.
 __device__ __forceinline__ float scale_reciprocal(float s) { return s == 0.0f ? 0.0f : __frcp_rn(s); }
 
 __device__ __forceinline__ int clamp127(int q) { return q > 127 ? 127 : (q < -127 ? -127 : q); }
+
+// Bytes whose bit is set in the low four bits of `bits` -> 0xFF, others 0.
+__device__ __forceinline__ uint32_t byte_mask4(uint32_t bits) {
+  return ((((bits & 0xFu) * 0x00204081u) & 0x01010101u) * 0xFFu);
+}
 
 // Eight halves packed in a uint4 -> their eight codes packed in a uint2.
 // Lanes whose bit is set in `skip` get code 0.  The eight codes are formed
 // independently (no branch per element); the rare near-tie elements are
 // redone with the division afterwards.
 __device__ __forceinline__ uint2 quant8(const uint4 v, float s, float inv, uint32_t skip) {
+  constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
   const uint32_t w[4] = {v.x, v.y, v.z, v.w};
   float x[8];
-  int q[8];
-  uint32_t near = 0;
+  uint32_t tb[8];
+  bool near = false;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w[j]));
+    x[2 * j] = f.x;
+    x[2 * j + 1] = f.y;
+  }
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
-    x[i] = half_bits_to_float(w[i >> 1] >> ((i & 1) * 16));
-    const float a = x[i] * inv;
-    const float r = rintf(a);
-    near |= (fabsf(a - r) >= 0.5f - 0x1p-12f ? 1u : 0u) << i;
-    q[i] = clamp127(__float2int_rn(r));
+    const float t = __fmaf_rn(x[i], inv, kMagic);
+    const float d = __fmaf_rn(x[i], inv, -__fsub_rn(t, kMagic));
+    near |= !(fabsf(d) < 0.5f - 0x1p-12f);
+    tb[i] = __float_as_uint(t);
   }
-  near &= ~skip;
+  uint32_t lo = __byte_perm(__byte_perm(tb[0], tb[1], 0x0040), __byte_perm(tb[2], tb[3], 0x0040), 0x5410);
+  uint32_t hi = __byte_perm(__byte_perm(tb[4], tb[5], 0x0040), __byte_perm(tb[6], tb[7], 0x0040), 0x5410);
   if (near) {
+    // redo the near-tie lanes with the division
 #pragma unroll
-    for (int i = 0; i < 8; ++i)
-      if ((near >> i) & 1u) q[i] = quant_code(x[i], s);
+    for (int i = 0; i < 8; ++i) {
+      const float t = __uint_as_float(tb[i]);
+      const float d = __fmaf_rn(x[i], inv, -__fsub_rn(t, kMagic));
+      if (!((skip >> i) & 1u) && !(fabsf(d) < 0.5f - 0x1p-12f)) {
+        const uint32_t q = static_cast<uint32_t>(quant_code(x[i], s)) & 0xFFu;
+        const int sh = (i & 3) * 8;
+        if (i < 4)
+          lo = (lo & ~(0xFFu << sh)) | (q << sh);
+        else
+          hi = (hi & ~(0xFFu << sh)) | (q << sh);
+      }
+    }
   }
-  uint32_t out[2] = {0u, 0u};
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const int qi = ((skip >> i) & 1u) ? 0 : q[i];
-    out[i >> 2] |= (static_cast<uint32_t>(qi) & 0xFFu) << ((i & 3) * 8);
+  if (skip) {
+    lo &= ~byte_mask4(skip);
+    hi &= ~byte_mask4(skip >> 4);
   }
-  return make_uint2(out[0], out[1]);
+  return make_uint2(lo, hi);
 }
 
 // ---------------------------------------------------------------------------
@@ -105,25 +136,60 @@ __device__ __forceinline__ uint2 quant8_codes(const uint4 v, float s, float inv,
     return quant8(v, s, inv, skip);
 }
 
-// max |x| over the lanes of eight halves whose bit is clear in `skip`.
+// max |x| over the lanes of eight halves whose bit is clear in `skip`, merged
+// into m.  The maximum of fp16 magnitudes is one of them, so it is taken in
+// half2 (NaN lanes are ignored, as by fmaxf) and widened once.
 __device__ __forceinline__ float absmax8(const uint4 v, uint32_t skip, float m) {
+  uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  if (skip) {
+    // a skipped lane becomes +0 (bits 0x0000)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const uint32_t b = (skip >> (2 * j)) & 3u;
+      w[j] &= ((b & 1u) ? 0xFFFF0000u : 0xFFFFFFFFu) & ((b & 2u) ? 0x0000FFFFu : 0xFFFFFFFFu);
+    }
+  }
+  const __half2 h0 = __hmax2(__habs2(*reinterpret_cast<const __half2*>(&w[0])),
+                             __habs2(*reinterpret_cast<const __half2*>(&w[1])));
+  const __half2 h1 = __hmax2(__habs2(*reinterpret_cast<const __half2*>(&w[2])),
+                             __habs2(*reinterpret_cast<const __half2*>(&w[3])));
+  const float2 f = __half22float2(__hmax2(h0, h1));
+  return fmaxf(m, fmaxf(f.x, f.y));
+}
+
+// The smallest fp16 value >= tau (+inf above the largest finite half): for an
+// fp16 x, |x| >= tau (binary32) exactly when |x| >= this value (fp16).
+__device__ __forceinline__ __half2 tau_half2(float tau) {
+  const __half h = __float2half_ru(tau);
+  return __halves2half2(h, h);
+}
+
+// |x| >= tau for the eight halves, as four words of two 16-bit lane masks
+// (0xFFFF where true; NaN never is).  OR-ing these over rows and turning the
+// result into bits once (mask_bits) is the cheap way to detect over many rows.
+struct Mask8 {
+  uint32_t m[4];
+};
+
+__device__ __forceinline__ void outlier_mask8_or(const uint4 v, __half2 tau2, Mask8& acc) {
   const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    if ((skip >> i) & 1u) continue;
-    m = fmaxf(m, fabsf(half_bits_to_float(w[i >> 1] >> ((i & 1) * 16))));
-  }
-  return m;
+  for (int j = 0; j < 4; ++j) acc.m[j] |= __hge2_mask(__habs2(*reinterpret_cast<const __half2*>(&w[j])), tau2);
+}
+
+// Bit i set iff lane i of the masks is set.
+__device__ __forceinline__ uint32_t mask_bits(const Mask8& a) {
+  uint32_t r = 0;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) r |= ((a.m[j] & 1u) << (2 * j)) | (((a.m[j] >> 16) & 1u) << (2 * j + 1));
+  return r;
 }
 
 // Bit i set iff |lane i| >= tau.
-__device__ __forceinline__ uint32_t outlier_mask8(const uint4 v, float tau) {
-  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-  uint32_t m = 0;
-#pragma unroll
-  for (int i = 0; i < 8; ++i)
-    m |= (fabsf(half_bits_to_float(w[i >> 1] >> ((i & 1) * 16))) >= tau ? 1u : 0u) << i;
-  return m;
+__device__ __forceinline__ uint32_t outlier_mask8(const uint4 v, __half2 tau2) {
+  Mask8 a = {{0u, 0u, 0u, 0u}};
+  outlier_mask8_or(v, tau2, a);
+  return mask_bits(a);
 }
 
 __device__ __forceinline__ float warp_max(float v) {

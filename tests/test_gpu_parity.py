@@ -134,6 +134,64 @@ def test_detect_edge_values(L, oracle, path):
     assert host(sx)[3] == 0.0
 
 
+@pytest.mark.parametrize("path", [1, 2])
+def test_detect_thresholds_between_halves(L, oracle, path):
+    """Thresholds that are not fp16 values (between two halves, below the
+    smallest subnormal, above the largest finite half, negative): the test
+    |x| >= tau is the binary32 one."""
+    pos = np.arange(0, 0x7c00, dtype=np.uint16)
+    vals = np.concatenate([pos, pos | 0x8000]).view(np.float16)
+    T = 16
+    X = np.ascontiguousarray(vals[np.random.default_rng(3).permutation(vals.size)][: T * 3968].reshape(T, 3968))
+    for tau in (6.0001, float(np.nextafter(np.float32(6.0), np.float32(0))), 1e-8, 70000.0, 65504.0, -1.0,
+                0.0):
+        flag = oracle.detect_outliers(X, tau)
+        idx_o = oracle.compact(flag)
+        Xq_o, sx_o = oracle.quantize_activations(X, flag)
+        Xq, sx, idx = activation_stages(L, X, tau, path)
+        assert_equal(host(idx), idx_o, f"idx tau={tau}")
+        assert_equal(host(sx).view(np.uint32), sx_o.view(np.uint32), f"sx tau={tau}")
+        assert_equal(host(Xq), Xq_o, f"Xq tau={tau}")
+    ok_status(L)
+
+
+def every_fp16_rows(K, seed):
+    """Every finite fp16 value (both zeros included) once, shuffled into rows
+    of K, plus rows that put every value below a chosen row maximum under that
+    maximum's scale (so small codes and every rounding boundary are reached)."""
+    pos = np.arange(0, 0x7c00, dtype=np.uint16)
+    vals = np.concatenate([pos, pos | 0x8000]).view(np.float16)
+    rng = np.random.default_rng(seed)
+    rows = [vals[rng.permutation(vals.size)][: (vals.size // K) * K].reshape(-1, K)]
+    for amax in (np.float16(127 * 2.0 ** -7), np.float16(0.37), np.float16(1.0), np.float16(5.99),
+                 np.float16(127.0), np.float16(3000.0)):
+        below = vals[np.abs(vals.astype(np.float32)) <= np.float32(amax)]
+        take = below[rng.permutation(below.size)][: (below.size // (K - 1)) * (K - 1)].reshape(-1, K - 1)
+        take = take[:64]
+        rows.append(np.concatenate([take, np.full((take.shape[0], 1), amax, np.float16)], axis=1))
+    return np.ascontiguousarray(np.concatenate(rows))
+
+
+@pytest.mark.parametrize("path", [1, 2])
+def test_codes_every_fp16_value(L, oracle, path):
+    """Each finite fp16 value as an activation and as a weight element, under
+    many row scales, tau = inf (every column regular): the codes and scales
+    agree bit for bit with the oracle's IEEE quotient, rounded half to even."""
+    X = every_fp16_rows(256, seed=5 + path)
+    rows = [X[i:i + 16] for i in range(0, X.shape[0], 16)] if path == 1 else [X]
+    for Xr in rows:
+        Xq, sx, _ = activation_stages(L, np.ascontiguousarray(Xr), float("inf"), path)
+        Xq_o, sx_o = oracle.quantize_activations(Xr, np.zeros(Xr.shape[1], np.uint8))
+        assert_equal(host(sx).view(np.uint32), sx_o.view(np.uint32), "sx")
+        assert_equal(host(Xq), Xq_o, "Xq")
+    Wq, sw = L.llmint8_quantize_weight(dev(X))
+    Wq_o, sw_o = oracle.quantize_weight(X)
+    torch.cuda.synchronize()
+    assert_equal(host(sw).view(np.uint32), sw_o.view(np.uint32), "Wscale")
+    assert_equal(host(Wq), Wq_o, "Wq")
+    ok_status(L)
+
+
 def near_tie_rows(rng, nrows, K):
     """Rows of fp16 values whose binary32 quotient x/s lies within 2^-12 of a
     half-integer (or on it), s = max|row| / 127: the band where a
