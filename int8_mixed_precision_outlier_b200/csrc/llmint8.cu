@@ -289,8 +289,11 @@ int launch_prep(const Layout& L, const uint16_t* X, int T, int K, const uint16_t
     return e == cudaSuccess ? LLMINT8_OK : LLMINT8_ERR_CUDA;
   }
   float* rowmax = reinterpret_cast<float*>(ws + L.rowmax);
-  e = launch_ex(detect_kernel, dim3(L.nstrips * kDetectCluster), dim3(kPrepThreads), 0, st, true, kDetectCluster, X,
-                T, K, tau, L.rows_per_cta, flags, L.Kw, rowmax, L.nstrips);
+  // up to 16 rows per thread (T <= 2048): the rows stay in registers between the two passes
+  const int rpt = (L.rows_per_cta + 15) / 16;
+  auto detect = rpt <= 4 ? detect_kernel<4> : rpt <= 16 ? detect_kernel<16> : detect_kernel<0>;
+  e = launch_ex(detect, dim3(L.nstrips * kDetectCluster), dim3(kPrepThreads), 0, st, true, kDetectCluster, X, T, K,
+                tau, L.rows_per_cta, flags, L.Kw, rowmax, L.nstrips);
   if (e != cudaSuccess) return LLMINT8_ERR_CUDA;
   const int gather_ctas = W ? (N + kWoRowsPerCta - 1) / kWoRowsPerCta
                           : cs.slot ? (N + kStoreRowsPerCta - 1) / kStoreRowsPerCta : 0;

@@ -100,7 +100,9 @@ __global__ void __launch_bounds__(kPrepThreads) quantize_weight_kernel(
 // ---------------------------------------------------------------------------
 constexpr int kDetectCols = 128;
 constexpr int kDetectCluster = 8;
-
+// KEEP > 0: each thread's rows (at most KEEP) stay in registers between the
+// two passes; KEEP = 0 reads them again.
+template <int KEEP>
 __global__ void __launch_bounds__(kPrepThreads) detect_kernel(const uint16_t* __restrict__ X, int T, int K,
                                                               float tau, int rpc, uint32_t* __restrict__ flags,
                                                               int Kw, float* __restrict__ rowmax, int nstrips) {
@@ -122,7 +124,18 @@ __global__ void __launch_bounds__(kPrepThreads) detect_kernel(const uint16_t* __
   constexpr int U = 8;
   const __half2 tau2 = tau_half2(tau);
   Mask8 acc = {{0u, 0u, 0u, 0u}};
-  if (live) {
+  uint4 kv[KEEP > 0 ? KEEP : 1];  // this thread's rows t0 + rr + 16 i, all loads in flight at once
+  if constexpr (KEEP > 0) {
+#pragma unroll
+    for (int i = 0; i < KEEP; ++i) {
+      const int t = t0 + rr + 16 * i;
+      kv[i] = (live && t < t1) ? __ldg(reinterpret_cast<const uint4*>(base + static_cast<int64_t>(t) * K))
+                               : make_uint4(0u, 0u, 0u, 0u);
+    }
+#pragma unroll
+    for (int i = 0; i < KEEP; ++i)  // only loaded rows (a zero fill passes |x| >= tau for tau <= 0)
+      if (live && t0 + rr + 16 * i < t1) outlier_mask8_or(kv[i], tau2, acc);
+  } else if (live) {
     int t = t0 + rr;
     for (; t + 16 * (U - 1) < t1; t += 16 * U) {
       uint4 v[U];
@@ -154,22 +167,33 @@ __global__ void __launch_bounds__(kPrepThreads) detect_kernel(const uint16_t* __
   // the strip maxima of this CTA's rows over the regular columns
   const uint32_t skip = live ? (fw >> ((c & 3) * 8)) & 0xFFu : 0xFFu;
   const int rounds = (t1 - t0 + 15) / 16;  // uniform over the CTA (the shuffles need whole half-warps)
-  for (int i0 = 0; i0 < rounds; i0 += U) {
-    uint4 v[U];
+  if constexpr (KEEP > 0) {
 #pragma unroll
-    for (int u = 0; u < U; ++u) {
-      const int t = t0 + rr + 16 * (i0 + u);
-      v[u] = (live && i0 + u < rounds && t < t1)
-                 ? __ldg(reinterpret_cast<const uint4*>(base + static_cast<int64_t>(t) * K))
-                 : make_uint4(0u, 0u, 0u, 0u);
-    }
-#pragma unroll
-    for (int u = 0; u < U; ++u) {
-      float m = absmax8(v[u], skip, 0.0f);
+    for (int i = 0; i < KEEP; ++i) {
+      float m = absmax8(kv[i], skip, 0.0f);
 #pragma unroll
       for (int o = 8; o >= 1; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-      const int t = t0 + rr + 16 * (i0 + u);
-      if (c == 0 && i0 + u < rounds && t < t1) rowmax[static_cast<int64_t>(t) * nstrips + strip] = m;
+      const int t = t0 + rr + 16 * i;
+      if (c == 0 && i < rounds && t < t1) rowmax[static_cast<int64_t>(t) * nstrips + strip] = m;
+    }
+  } else {
+    for (int i0 = 0; i0 < rounds; i0 += U) {
+      uint4 v[U];
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int t = t0 + rr + 16 * (i0 + u);
+        v[u] = (live && i0 + u < rounds && t < t1)
+                   ? __ldg(reinterpret_cast<const uint4*>(base + static_cast<int64_t>(t) * K))
+                   : make_uint4(0u, 0u, 0u, 0u);
+      }
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        float m = absmax8(v[u], skip, 0.0f);
+#pragma unroll
+        for (int o = 8; o >= 1; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+        const int t = t0 + rr + 16 * (i0 + u);
+        if (c == 0 && i0 + u < rounds && t < t1) rowmax[static_cast<int64_t>(t) * nstrips + strip] = m;
+      }
     }
   }
 }

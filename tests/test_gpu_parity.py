@@ -155,6 +155,19 @@ def test_detect_thresholds_between_halves(L, oracle, path):
     ok_status(L)
 
 
+@pytest.mark.parametrize("T,K", [(37, 1040), (520, 1040), (2100, 272), (129, 16)])
+def test_detect_nonpositive_threshold_ragged(L, oracle, T, K):
+    """tau <= 0 flags every column, and no more: K not a multiple of the
+    detection strip, row counts that leave the strip's scanners partly idle
+    (padding must never count as data)."""
+    X, _ = synth.make_activations(T, K, seed=T + K, n_dims=2, mag=(6.0, 60.0))
+    for tau in (0.0, -1.0):
+        Xq, sx, idx = activation_stages(L, X, tau, 2)
+        assert_equal(host(idx), np.arange(K, dtype=np.int32), f"idx tau={tau}")
+        assert not host(Xq).any() and not host(sx).any()
+    ok_status(L)
+
+
 def every_fp16_rows(K, seed):
     """Every finite fp16 value (both zeros included) once, shuffled into rows
     of K, plus rows that put every value below a chosen row maximum under that
