@@ -125,9 +125,16 @@ def source_digest() -> str:
     return h.hexdigest()[:16]
 
 
+def traffic_key(workload: str, tau: float) -> str:
+    """The workload's name in profiles/traffic.txt: with '@tau' when the call
+    runs at a threshold other than the default (the 70B sweep)."""
+    return workload if tau == THRESHOLD else f"{workload}@{tau:g}"
+
+
 def recorded_traffic(workload: str, kernel: str):
-    """dram bytes per launch of `kernel` on `workload` from profiles/traffic.txt
-    (lines: workload kernel source_digest bytes_per_launch), or None."""
+    """dram bytes per launch of `kernel` on `workload` (a traffic_key) from
+    profiles/traffic.txt (lines: workload kernel source_digest bytes_per_launch),
+    or None."""
     p = os.path.join(ROOT, "profiles", "traffic.txt")
     if not os.path.exists(p):
         return None
@@ -525,11 +532,10 @@ def prefill_roofline(wl: Workload, kern_ms: float, c: dict, peaks: dict, traffic
 
 def e2e_steps(wl: Workload, steps: int, warmup: int, flush, world: int = 1) -> dict:
     """The public call with host buffers: pinned H2D of X, the matmul, D2H of Y,
-    for every call of the step, captured once into a CUDA graph (the way a
-    decode loop drives the library) and replayed per step, so each step still
-    copies its inputs in and its results out.  Every rank runs it; the value is
-    all ranks' units over the slowest rank's time, and the copy bytes are the
-    whole job's."""
+    for every call of the step, issued as direct calls (capturing them into a
+    CUDA graph measured slower: 1105 against 1174 GB/s, the ten small copies of
+    a step dominate either way).  Every rank runs it; the value is all ranks'
+    units over the slowest rank's time, and the copy bytes are the whole job's."""
     import torch
     hx = [torch.from_numpy(c["host_X"]).pin_memory() for c in wl.calls]
     hy = [torch.empty(c["Y"].shape, dtype=torch.float16).pin_memory() for c in wl.calls]
@@ -540,14 +546,7 @@ def e2e_steps(wl: Workload, steps: int, warmup: int, flush, world: int = 1) -> d
             wl.call(c)
             y.copy_(c["Y"], non_blocking=True)
 
-    run()
-    torch.cuda.synchronize()
-    g = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g):
-        run()
-    torch.cuda.synchronize()
-    total_ms, _ = time_steps(wl, steps, warmup, world, flush, run=g.replay)
-    del g
+    total_ms, _ = time_steps(wl, steps, warmup, world, flush, run=run)
     t_max = reduce_max(total_ms, world)
     units = reduce_sum((wl.bytes_per_step if wl.unit == "GB/s" else wl.ops_per_step) * steps, world)
     value = units / (t_max * 1e-3) / (1e9 if wl.unit == "GB/s" else 1e12)
@@ -556,7 +555,7 @@ def e2e_steps(wl: Workload, steps: int, warmup: int, flush, world: int = 1) -> d
     return {"value": round(value, 2), "unit": wl.unit,
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
             "ms_per_step": round(t_max / steps, 5),
-            "how": "pinned H2D of X, llmint8 call, D2H of Y for each call of the step, one CUDA graph replay per step"}
+            "how": "pinned H2D of X, llmint8 call, D2H of Y for each call of the step, direct calls"}
 
 
 # ----------------------------------------------------------------- CPU oracle
@@ -724,11 +723,13 @@ def also_entry(name, variant, tau, device, peaks, flush, steps, oracle_budget_s)
     if w2.unit == "GB/s":
         cold_ms, cold_algo = time_cold_units(w2, 10, flush)
         entry["roofline"] = decode_roofline(w2, ms / steps, cold_ms, cold_algo, peaks,
-                                            traffic=recorded_traffic(name, main_kernel_name(w2)))
+                                            traffic=recorded_traffic(traffic_key(name, c["tau"]),
+                                                                     main_kernel_name(w2)))
     else:
         km, _ = time_cold_units(w2, 10, flush)
         b2b = time_back_to_back(w2, flush) if variant == "llmint8" else None
-        entry["roofline"] = prefill_roofline(w2, km, c, peaks, traffic=recorded_traffic(name, main_kernel_name(w2)),
+        entry["roofline"] = prefill_roofline(w2, km, c, peaks,
+                                             traffic=recorded_traffic(traffic_key(name, c["tau"]), main_kernel_name(w2)),
                                              b2b_ms=b2b)
         call_tops = w2.ops_per_step / (ms / steps * 1e-3) / 1e12   # the whole call, graph-replayed
         entry["call_roofline_frac"] = round(call_tops / entry["roofline"]["peak"], 4)
@@ -768,7 +769,7 @@ def run_ours(args):
     value = units / (t_max * 1e-3) / (1e9 if wl.unit == "GB/s" else 1e12)
     status = L.llmint8_sync_status()
     cold_ms, cold_algo = time_cold_units(wl, 10, flush)
-    traffic = recorded_traffic(args.workload, main_kernel_name(wl))
+    traffic = recorded_traffic(traffic_key(args.workload, wl.calls[0]["tau"]), main_kernel_name(wl))
     if wl.unit == "GB/s":
         roof = decode_roofline(wl, total_ms / args.steps, cold_ms, cold_algo, peaks, traffic=traffic)
     else:

@@ -115,23 +115,60 @@ __device__ __forceinline__ uint32_t e4m3_code(float v, float s) {
   return static_cast<uint32_t>(__nv_cvt_float_to_fp8(__fdiv_rn(v, s), __NV_SATFINITE, __NV_E4M3));
 }
 
-// Eight halves -> eight E4M3 codes (lanes set in `skip` get 0).
-__device__ __forceinline__ uint2 quant8_e4m3(const uint4 v, float s, uint32_t skip) {
+// Eight halves -> eight E4M3 codes (lanes set in `skip` get 0), without a
+// division in the common case.  With inv = fl(1/s) and a = fl(x * inv):
+//   |a - x/s| <= 2^-23 |x/s| (two roundings) and |fl(x/s) - x/s| <= 2^-24 |x/s|,
+// so fl(x/s) lies strictly between fl(a (1 - 2^-20)) and fl(a (1 + 2^-20))
+// (each still at least 2^-21 |a| away from a).  The conversion (round to
+// nearest even, saturating) is monotonic, so when it gives one code for both
+// ends it gives that code for fl(x/s) too; otherwise (a value next to a
+// rounding point of E4M3) the lane takes the IEEE division.  Pairs of lanes
+// go through the two-float conversion.
+__device__ __forceinline__ uint2 quant8_e4m3(const uint4 v, float s, float inv, uint32_t skip) {
+  if (s == 0.0f) return make_uint2(0u, 0u);
+  constexpr float kDown = 1.0f - 0x1p-20f, kUp = 1.0f + 0x1p-20f;
   const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-  uint32_t out[2] = {0u, 0u};
+  uint32_t pair[4];
+  uint32_t differ = 0;  // bit i: lane i's two ends convert differently
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const uint32_t c = ((skip >> i) & 1u) ? 0u : e4m3_code(half_bits_to_float(w[i >> 1] >> ((i & 1) * 16)), s);
-    out[i >> 2] |= c << ((i & 3) * 8);
+  for (int j = 0; j < 4; ++j) {
+    const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w[j]));
+    const float a0 = __fmul_rn(f.x, inv), a1 = __fmul_rn(f.y, inv);
+    const uint32_t lo = __nv_cvt_float2_to_fp8x2(make_float2(__fmul_rn(a0, kDown), __fmul_rn(a1, kDown)),
+                                                 __NV_SATFINITE, __NV_E4M3);
+    const uint32_t hi = __nv_cvt_float2_to_fp8x2(make_float2(__fmul_rn(a0, kUp), __fmul_rn(a1, kUp)),
+                                                 __NV_SATFINITE, __NV_E4M3);
+    const uint32_t d = lo ^ hi;
+    differ |= ((d & 0xFFu) ? 1u : 0u) << (2 * j) | ((d & 0xFF00u) ? 1u : 0u) << (2 * j + 1);
+    pair[j] = lo;
   }
-  return make_uint2(out[0], out[1]);
+  uint32_t lo32 = (pair[0] & 0xFFFFu) | (pair[1] << 16);
+  uint32_t hi32 = (pair[2] & 0xFFFFu) | (pair[3] << 16);
+  differ &= ~skip;
+  if (differ) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      if (!((differ >> i) & 1u)) continue;
+      const uint32_t c = e4m3_code(half_bits_to_float(w[i >> 1] >> ((i & 1) * 16)), s);
+      const int sh = (i & 3) * 8;
+      if (i < 4)
+        lo32 = (lo32 & ~(0xFFu << sh)) | (c << sh);
+      else
+        hi32 = (hi32 & ~(0xFFu << sh)) | (c << sh);
+    }
+  }
+  if (skip) {
+    lo32 &= ~byte_mask4(skip);
+    hi32 &= ~byte_mask4(skip >> 4);
+  }
+  return make_uint2(lo32, hi32);
 }
 
-// Codes of either format; `inv` (= fl(1/s)) is used by the int8 codes only.
+// Codes of either format (inv = fl(1/s), 0 for s == 0).
 template <bool FP8>
 __device__ __forceinline__ uint2 quant8_codes(const uint4 v, float s, float inv, uint32_t skip) {
   if constexpr (FP8)
-    return quant8_e4m3(v, s, skip);
+    return quant8_e4m3(v, s, inv, skip);
   else
     return quant8(v, s, inv, skip);
 }

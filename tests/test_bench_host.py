@@ -65,6 +65,17 @@ def test_recorded_traffic_needs_the_current_digest(tree):
     assert bench.recorded_traffic("13b_up", "gemm_pair_kernel") is None
 
 
+def test_traffic_key_names_the_threshold_sweep(tree):
+    d = bench.source_digest()
+    (tree / "profiles" / "traffic.txt").write_text(
+        f"70b_up gemm_pair_kernel {d} 605212672\n70b_up@4 gemm_pair_kernel {d} 1401019904\n"
+        f"70b_up@inf gemm_pair_kernel {d} 584742656\n", encoding="utf-8")
+    assert bench.traffic_key("70b_up", bench.THRESHOLD) == "70b_up"
+    assert bench.recorded_traffic(bench.traffic_key("70b_up", 4.0), "gemm_pair_kernel") == 1401019904.0
+    assert bench.recorded_traffic(bench.traffic_key("70b_up", float("inf")), "gemm_pair_kernel") == 584742656.0
+    assert bench.recorded_traffic(bench.traffic_key("70b_up", 6.0), "gemm_pair_kernel") == 605212672.0
+
+
 def test_shrink_sample_recounts_bytes_and_ops():
     T, N, K, n_out = 4, 1000, 256, 3
     X = np.zeros((T, K), np.float16)
