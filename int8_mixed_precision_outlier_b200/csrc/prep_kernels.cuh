@@ -397,27 +397,20 @@ __global__ void __launch_bounds__(kQuantThreads, 8) quant_gather_kernel(
       __syncthreads();  // the previous window's indices have been read
       list_outliers(sflags, wpre, Kw, win, min(nO, win + kGatherIdxCap), si);
       __syncthreads();
+      // thread i takes column jj = i (+ 128 ...) of the window, 8 rows at a time
       const int width = min(opad - win, kGatherIdxCap);
-      const int total = rows * width;
       constexpr int UG = 8;
-      for (int base = threadIdx.x; base < total; base += UG * kQuantThreads) {
-        uint16_t v[UG];
+      for (int jj = static_cast<int>(threadIdx.x); jj < width; jj += kQuantThreads) {
+        const bool real = win + jj < nO;  // past |O|: padding, zeros
+        const int k = real ? si[jj] : 0;
+        for (int r0 = 0; r0 < rows; r0 += UG) {
+          uint16_t v[UG];
 #pragma unroll
-        for (int u = 0; u < UG; ++u) {
-          const int e = base + u * kQuantThreads;
-          v[u] = 0;
-          if (e < total) {
-            const int rr = e / width, jj = e - rr * width;
-            if (win + jj < nO) v[u] = __ldg(W + (n0 + rr) * K + si[jj]);
-          }
-        }
+          for (int u = 0; u < UG; ++u)
+            v[u] = (real && r0 + u < rows) ? __ldg(W + (n0 + r0 + u) * K + k) : uint16_t(0);
 #pragma unroll
-        for (int u = 0; u < UG; ++u) {
-          const int e = base + u * kQuantThreads;
-          if (e < total) {
-            const int rr = e / width, jj = e - rr * width;
-            Wo[(n0 + rr) * ldo + win + jj] = v[u];
-          }
+          for (int u = 0; u < UG; ++u)
+            if (r0 + u < rows) Wo[(n0 + r0 + u) * ldo + win + jj] = v[u];
         }
       }
     }
