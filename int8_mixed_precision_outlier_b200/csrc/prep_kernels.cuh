@@ -91,12 +91,14 @@ __global__ void __launch_bounds__(kPrepThreads) quantize_weight_kernel(
 // rowmax[t * nstrips + s] (the row's absmax is the maximum of these).
 // A cluster of kDetectCluster CTAs owns a strip; CTA r scans rows
 // [r*rpc, (r+1)*rpc).  Thread (c = tid % 16, rr = tid / 16) reads the 16
-// bytes of chunk c in every 16th row, 8 rows in flight, and ORs 16-bit lane
-// masks (the bits are formed once at the end).  Every CTA sends its four
-// words to every CTA of the cluster (distributed shared memory), so after one
-// cluster barrier each holds the strip's final flags: the first CTA writes
-// them, and every CTA reads its rows again (from L1 / L2) for their maxima
-// over the unflagged columns, reduced over the 16 lanes of a row.
+// bytes of chunk c in every 16th row and ORs 16-bit lane masks (the bits are
+// formed once at the end).  With KEEP > 0 a thread's rows (at most KEEP) are
+// loaded all at once and stay in registers; with KEEP = 0 they are streamed
+// 8 at a time and read again (from L1 / L2) for the second pass.  Every CTA
+// sends its four words to every CTA of the cluster (distributed shared
+// memory), so after one cluster barrier each holds the strip's final flags:
+// the first CTA writes them, and every CTA takes its rows' maxima over the
+// unflagged columns, reduced over the 16 lanes of a row.
 // ---------------------------------------------------------------------------
 constexpr int kDetectCols = 128;
 constexpr int kDetectCluster = 8;
